@@ -1,0 +1,57 @@
+"""Pin sensitivity: plant one plausible mistake at a time in a copy of the oracle's
+C source (on the CPU), build it, and require that at least one pin fails.  The
+shipped oracle is never modified."""
+import os
+import tempfile
+
+import pytest
+
+import oracle
+from tests import oracle_pins as pins
+
+with open(oracle.SOURCE) as _fh:
+    _SRC = _fh.read()
+
+# (name, original text, planted mistake)
+MUTANTS = [
+    ("summary_min_flipped", "if (x < lo) lo = x;", "if (x > lo) lo = x;"),
+    ("bound_takes_min", "u += (lo > hi) ? lo : hi;", "u += (lo < hi) ? lo : hi;"),
+    ("bound_only_max_side", "u += (lo > hi) ? lo : hi;", "u += hi;"),
+    ("group_sum_dropped", "total += u;", "total = u;"),
+    ("wrong_head_row", "double lo = q[h * d + c] * smin", "double lo = q[c] * smin"),
+    ("tie_to_higher_index", "return ia < ib;", "return ia > ib;"),
+    ("ema_alpha_beta_swapped", "double decayed = alpha * e[b];", "double decayed = beta * e[b];"),
+    ("ema_no_decay", "double decayed = alpha * e[b];", "double decayed = e[b];"),
+    ("attention_scale_dropped", "double p = exp(scale * dot_q_k(q, k + (size_t)t * d, d) - m);",
+     "double p = exp(dot_q_k(q, k + (size_t)t * d, d) - m);"),
+    ("attention_tail_token_dropped",
+     "int t0 = blocks[i] * bs, t1 = t0 + bs < n ? t0 + bs : n;\n        for (int t = t0; t < t1; ++t) {\n            double p",
+     "int t0 = blocks[i] * bs, t1 = t0 + bs < n ? t0 + bs : n - 1;\n        for (int t = t0; t < t1; ++t) {\n            double p"),
+    ("merge_unweighted", "double w = exp(m[j] - ms);", "double w = 1.0;"),
+    ("merge_lse_without_max", "*lse = ms + log(ls);", "*lse = log(ls);"),
+    ("missed_set_inverted", "if (!contains(pred, npred, sel[i])) missed[nm++]",
+     "if (contains(pred, npred, sel[i])) missed[nm++]"),
+    ("partial_no_max_shift", "double p = exp(scale * dot_q_k(q, k + (size_t)t * d, d) - mm);",
+     "double p = exp(scale * dot_q_k(q, k + (size_t)t * d, d));"),
+]
+
+
+@pytest.mark.parametrize("name,orig,bad", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, orig, bad):
+    assert _SRC.count(orig) >= 1, f"mutation anchor for {name} not found"
+    src = _SRC.replace(orig, bad, 1)
+    with tempfile.TemporaryDirectory() as tmp:
+        c = os.path.join(tmp, "mutant.c")
+        so = os.path.join(tmp, "libmutant.so")
+        with open(c, "w") as fh:
+            fh.write(src)
+        oracle.build(source=c, output=so, force=True)
+        o = oracle.Oracle(so)
+        failed = []
+        for check in pins.ALL_CHECKS:
+            try:
+                check(o)
+            except AssertionError:
+                failed.append(check.__name__)
+                break
+        assert failed, f"no pin caught the planted mistake {name}"
