@@ -1,0 +1,84 @@
+// prr_params.h -- kernel parameter block and workspace layout shared by the host
+// launchers and the device kernels of the PRR decode step.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+namespace prr {
+
+// Device status codes written (first error wins) into the workspace status word.
+enum : int {
+  kDevOk = 0,
+  kDevBadSeqLen = 1,      // seq_lens[b] < 1 or > cap_tokens
+  kDevBadPred = 2,         // predicted list not strictly ascending / out of range
+  kDevBadMissed = 3,       // missed list entry out of range
+  kDevWaitTimeout = 4,     // a bounded mbarrier wait gave up
+  kDevBadRange = 5,        // summary update range outside [0, cap_tokens]
+};
+
+// A bounded wait gives up after this long (one second).
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+// Merge tickets: the contributions of one (sequence, KV head) add up to this value
+// exactly once, and whoever brings the counter there runs the LSE merge.
+constexpr unsigned kMergeTarget = 1u << 30;
+
+enum : int { MODE_STANDALONE = 0, MODE_STEP = 1 };
+
+// Byte offsets inside the caller-owned workspace (all 256-byte aligned).
+struct WsLayout {
+  size_t status;     // int32 status word
+  size_t sel_cnt;    // uint32 [units] chunk tickets of the selection kernel
+  size_t merge_cnt;  // uint32 [units] merge tickets
+  size_t cand;       // uint64 [units][max_chunks][list_len] per-chunk top lists
+  size_t rm;         // float [units*G][K] repair partial max (base-2 logits)
+  size_t rl;         // float [units*G][K] repair partial sum
+  size_t rO;         // float [units*G][K][d] repair partial numerator
+  size_t total;
+  int max_chunks;
+  int list_len;
+};
+
+struct Params {
+  // shape
+  int B, Hq, Hkv, G, d, bs, cap, K, P, maxnb, units;
+  float scale_log2;  // softmax scale * log2(e): logits are handled in base 2
+  double alpha;      // EMA decay
+  int mode;
+  // selection geometry
+  int chunk_blocks;  // blocks per selection CTA (multiple of 32)
+  int nchunks;       // selection CTAs per unit
+  int list_len;      // 32 * keys per lane
+  // caller buffers (any may be null when the kernel does not use it)
+  const uint16_t* q;        // [B][Hq][d] bf16
+  const uint16_t* kc;       // [B][Hkv][cap][d] bf16
+  const uint16_t* vc;       // [B][Hkv][cap][d] bf16
+  const int* seq_lens;      // [B]
+  uint16_t* summ;           // [B][Hkv][maxnb][2][d] bf16 (min row, max row)
+  double* ema;              // [B][Hkv][maxnb]
+  const int* pred;          // [B][Hkv][P]  Pred_t
+  int* pred_next;           // [B][Hkv][P]  Pred_{t+1}
+  int* sel;                 // [B][Hkv][K]
+  int* missed;              // [B][Hkv][K]
+  int* n_missed;            // [B][Hkv]
+  uint8_t* keep;            // [B][Hkv][P]
+  float* pm;                // [B][Hq][P]
+  float* pl;                // [B][Hq][P]
+  float* pO;                // [B][Hq][P][d]
+  float* out;               // [B][Hq][d]
+  float* lse;               // [B][Hq]
+  // workspace views
+  int* status;
+  unsigned* sel_cnt;
+  unsigned* merge_cnt;
+  uint64_t* cand;
+  float* rm;
+  float* rl;
+  float* rO;
+  // summary update range (null: append of token seq_lens[b]-1)
+  const int* tok_begin;
+  const int* tok_end;
+};
+
+}  // namespace prr

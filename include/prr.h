@@ -1,0 +1,224 @@
+/*
+ * prr.h -- C ABI of the PRR decode-step library (sm_100a).
+ *
+ * PRR (Predict, Reuse, and Repair: Accelerating Dynamic Sparse Attention for
+ * Long-Context LLM Decoding) removes the wait between block selection and attention
+ * in dynamic sparse attention (DSA) decoding: an EMA of past selections predicts the
+ * blocks, attention over the predicted blocks runs while the true top-K is being
+ * selected, predicted blocks outside the true set are dropped, and the missed blocks
+ * are repaired and merged through online-softmax statistics.  The result equals plain
+ * top-K DSA attention whatever the prediction (PRR abstract; method summary;
+ * contributions (1)-(3)).
+ *
+ * Conventions shared by every entry point
+ *  - All array pointers are DEVICE pointers owned by the caller.  The library never
+ *    allocates, frees or synchronises device memory; only prr_get_device_status
+ *    synchronises (to read the status word back).
+ *  - bf16 arrays are passed as uint16_t bit patterns.
+ *  - Shapes (row-major, innermost last), with units = B*Hkv, G = Hq/Hkv,
+ *    maxnb = ceil(cap_tokens/bs):
+ *      q            [B][Hq][d]               bf16   query of the step
+ *      k_cache/v_cache [B][Hkv][cap_tokens][d] bf16 (16-byte aligned base)
+ *      seq_lens     [B]                      int32  tokens n in the cache, 1 <= n <= cap
+ *      summ         [B][Hkv][maxnb][2][d]    bf16   per block: min row then max row
+ *      ema          [B][Hkv][maxnb]          fp64   EMA state, starts at 0
+ *      pred, pred_next [B][Hkv][P]           int32  ascending block ids, -1 when empty
+ *      sel, missed  [B][Hkv][K]              int32  ascending block ids, -1 when empty
+ *      n_missed     [B][Hkv]                 int32
+ *      keep         [B][Hkv][P]              uint8  keep[j] = Pred_j in S_t
+ *      part_m, part_l [B][Hq][P]             fp32   speculative partials, one per slot
+ *      part_O       [B][Hq][P][d]            fp32
+ *      out          [B][Hq][d]               fp32   attention output
+ *      lse          [B][Hq]                  fp32   natural-log log-sum-exp of the logits
+ *    Partials use base-2 logits: part_m = max_i scale*log2(e)*q.k_i over the block,
+ *    part_l = sum_i 2^(logit_i - part_m), part_O = sum_i 2^(logit_i - part_m) v_i.
+ *  - Supported shapes: d in {64, 128}; bs in {64, 128}; 1 <= G <= 8; 1 <= K <= 128;
+ *    0 <= P <= 128; cap_tokens >= 1.  Others return PRR_ERR_SHAPE.
+ *  - Errors: argument and shape checks happen on the host before anything is
+ *    enqueued and return a prr_status.  A failed launch returns PRR_ERR_CUDA.
+ *    Problems that only the device can see (a seq_len out of range, a malformed
+ *    predicted list, a wait that timed out) set the status word in the workspace
+ *    (first error wins) and never trap; read it with prr_get_device_status.  After a
+ *    non-zero device status, re-initialise the workspace before the next call.
+ *  - Calls are asynchronous on the given stream(s).  Two calls that share a
+ *    workspace must not overlap on the GPU.
+ */
+#ifndef PRR_H
+#define PRR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PRR_OK = 0,
+  PRR_ERR_INVALID_ARG = 1,   /* null pointer or misaligned buffer */
+  PRR_ERR_SHAPE = 2,         /* unsupported or inconsistent dimensions */
+  PRR_ERR_CAPACITY = 3,      /* workspace smaller than prr_workspace_bytes() */
+  PRR_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+  PRR_ERR_DEVICE_STATUS = 5, /* prr_get_device_status found a device-side error */
+  PRR_ERR_TIMEOUT = 6        /* reserved: a bounded wait gave up (device code 4) */
+} prr_status;
+
+/* Device status codes (the value prr_get_device_status stores in *code). */
+#define PRR_DEV_OK 0
+#define PRR_DEV_BAD_SEQ_LEN 1  /* seq_lens[b] < 1 or > cap_tokens (that sequence is skipped) */
+#define PRR_DEV_BAD_PRED 2     /* predicted list entry out of range or not ascending */
+#define PRR_DEV_BAD_MISSED 3   /* missed list entry out of range */
+#define PRR_DEV_WAIT_TIMEOUT 4 /* a bounded wait for a TMA copy gave up */
+#define PRR_DEV_BAD_RANGE 5    /* summary update range outside [0, cap_tokens] */
+
+typedef struct {
+  int32_t B;          /* sequences */
+  int32_t Hq;         /* query heads */
+  int32_t Hkv;        /* KV heads (Hq % Hkv == 0) */
+  int32_t d;          /* head dim */
+  int32_t bs;         /* tokens per KV block */
+  int32_t cap_tokens; /* KV capacity per (sequence, KV head) */
+  int32_t K;          /* top-K blocks selected per (sequence, KV head) */
+  int32_t P;          /* speculation budget: predicted blocks per (sequence, KV head) */
+  double alpha;       /* EMA decay, 0 <= alpha <= 1 */
+  float scale;        /* softmax scale applied to q.k (usually 1/sqrt(d)) */
+} prr_dims;
+
+/* Buffers of one decode step (see the shapes above). */
+typedef struct {
+  const uint16_t* q;
+  const uint16_t* k_cache;
+  const uint16_t* v_cache;
+  const int32_t* seq_lens;
+  uint16_t* summ;
+  double* ema;
+  const int32_t* pred;  /* Pred_t (read) */
+  int32_t* pred_next;   /* Pred_{t+1} (written); must not alias pred */
+  int32_t* sel;
+  int32_t* missed;
+  int32_t* n_missed;
+  uint8_t* keep;
+  float* part_m;
+  float* part_l;
+  float* part_O;
+  float* out;
+  float* lse;
+} prr_step_buffers;
+
+/* Events of one decode step.  fork and join are required (any flags); the timing
+ * marks are optional (NULL to skip) and, when given, must be created with timing. */
+typedef struct {
+  cudaEvent_t fork;             /* recorded on select_stream, waited by spec_stream */
+  cudaEvent_t join;             /* recorded on spec_stream, waited by select_stream */
+  cudaEvent_t t_begin;          /* select_stream: before the summary update */
+  cudaEvent_t t_select_end;     /* select_stream: after selection */
+  cudaEvent_t t_repair_end;     /* select_stream: after repair */
+  cudaEvent_t t_ema_end;        /* select_stream: after the EMA predictor */
+  cudaEvent_t t_spec_begin;     /* spec_stream: before speculation */
+  cudaEvent_t t_spec_end;       /* spec_stream: after speculation */
+} prr_step_events;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int prr_version(void);
+
+/* Human-readable name of a status. */
+const char* prr_status_string(prr_status s);
+
+/* Bytes of workspace the calls below need for these dims (0 if the dims are
+ * unsupported).  The workspace holds the status word, selection and merge tickets,
+ * per-chunk candidate lists and the repair partials. */
+size_t prr_workspace_bytes(const prr_dims* dims);
+
+/* Zero-fill a workspace (required once before first use, and after a device error).
+ * The kernels leave their tickets re-armed, so steady-state calls need no reset. */
+prr_status prr_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronously read the workspace status word into *code (0 = no error). Returns
+ * PRR_OK if the code is 0, PRR_ERR_DEVICE_STATUS otherwise. */
+prr_status prr_get_device_status(const void* ws, int32_t* code);
+
+/* Write one new token per (sequence, KV head): k_new/v_new [B][Hkv][d] go to position
+ * seq_lens[b] of the caches, then seq_lens[b] is incremented (a full cache leaves
+ * seq_lens unchanged and sets PRR_DEV_BAD_SEQ_LEN). */
+prr_status prr_append_kv(const prr_dims* dims, const uint16_t* k_new, const uint16_t* v_new,
+                         int32_t* seq_lens, uint16_t* k_cache, uint16_t* v_cache, void* ws,
+                         cudaStream_t stream);
+
+/* Block key summaries (step a1).  For every sequence b and KV head, the summaries of
+ * the blocks touched by tokens [tok_begin[b], tok_end[b]) become the per-channel
+ * min/max over the block's tokens [block start, tok_end[b]): a range that starts
+ * inside a block is folded into the stored summary of that block's earlier tokens.
+ * tok_begin/tok_end are device int32 [B]; both NULL means "the token just appended":
+ * [seq_lens[b]-1, seq_lens[b]).  max_range_tokens bounds tok_end-tok_begin over all
+ * sequences (it sizes the grid).  Summary per Quest (Query-Aware Sparsity for
+ * Efficient Long-Context LLM Inference, in the PRR reference list). */
+prr_status prr_update_summaries(const prr_dims* dims, const uint16_t* k_cache,
+                                const int32_t* tok_begin, const int32_t* tok_end,
+                                const int32_t* seq_lens, int32_t max_range_tokens, uint16_t* summ,
+                                void* ws, cudaStream_t stream);
+
+/* Block scoring + top-K (steps a2-a3).  For each (b, KV head): the score of every
+ * block below nb = ceil(n/bs) is the sum over the G query heads of
+ * sum_c max(q_hc*min_bc, q_hc*max_bc); sel = the min(K, nb) best blocks under (score
+ * desc, block asc), written ascending; missed = sel \ pred ascending, n_missed its
+ * size; keep[j] = (pred[j] in sel).  A predicted slot is active when 0 <= pred[j] < nb.
+ * PRR abstract: the true selected set; method summary: repair only the missed blocks. */
+prr_status prr_select_topk(const prr_dims* dims, const uint16_t* q, const uint16_t* summ,
+                           const int32_t* seq_lens, const int32_t* pred, int32_t* sel,
+                           int32_t* missed, int32_t* n_missed, uint8_t* keep, void* ws,
+                           cudaStream_t stream);
+
+/* EMA predictor (step a4).  If sel is not NULL: e_b <- alpha*e_b + (1-alpha)*[b in sel]
+ * for every block b < nb (fp64, multiplies and add rounded separately).  Then
+ * pred_next = the min(P, nb) best blocks under (e desc, block asc), ascending, -1
+ * beyond.  With sel NULL the state is only read (the zero state predicts 0..P-1).
+ * PRR abstract and contribution (1): a lightweight EMA-based predictor. */
+prr_status prr_ema_predict(const prr_dims* dims, double* ema, const int32_t* sel,
+                           const int32_t* seq_lens, int32_t* pred_next, void* ws,
+                           cudaStream_t stream);
+
+/* Speculative attention (step a5): one (m, l, O) partial per active predicted slot j
+ * and query head, over the tokens of block pred[j] below n.  Inactive slots are left
+ * untouched.  PRR abstract: attention over the predicted blocks while selection is
+ * still running. */
+prr_status prr_speculate(const prr_dims* dims, const uint16_t* q, const uint16_t* k_cache,
+                         const uint16_t* v_cache, const int32_t* seq_lens, const int32_t* pred,
+                         float* part_m, float* part_l, float* part_O, void* ws,
+                         cudaStream_t stream);
+
+/* Repair + merge (step a6): attention partials over the missed blocks, then the LSE
+ * merge of the kept speculative partials (keep[j] = 1) and the repair partials:
+ *   m* = max m_j, l* = sum l_j 2^(m_j-m*), out = sum O_j 2^(m_j-m*) / l*,
+ *   lse = (m* + log2 l*) ln 2.
+ * The speculative partials must come from prr_speculate on the same pred and q.
+ * PRR method summary and contribution (3): fold the missed blocks into the partial
+ * state with online-softmax statistics, no recomputation. */
+prr_status prr_repair_merge(const prr_dims* dims, const uint16_t* q, const uint16_t* k_cache,
+                            const uint16_t* v_cache, const int32_t* seq_lens,
+                            const int32_t* missed, const int32_t* n_missed, const uint8_t* keep,
+                            const int32_t* pred, const float* part_m, const float* part_l,
+                            const float* part_O, float* out, float* lse, void* ws,
+                            cudaStream_t stream);
+
+/* One full decode step (a1-a7) after the caller appended the step's token:
+ *   select_stream: summary update -> selection -> repair -> EMA predictor
+ *   spec_stream:   speculation over buf->pred (runs concurrently with selection)
+ * Whichever of selection, speculation and repair finishes a (sequence, KV head) last
+ * runs its LSE merge, so no kernel waits for another.  On return the work is enqueued;
+ * select_stream waits for spec_stream at the end (event join), so completion of
+ * select_stream means the step is done.  Selection, repair and the summary update run
+ * at the highest stream priority; speculation and the predictor at the lowest.  The
+ * caller swaps pred/pred_next between steps.  Capturable in a CUDA graph (no
+ * allocation, no synchronisation).  PRR method summary: speculation overlaps
+ * selection; the speculative budget keeps it off the critical path. */
+prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* buf, void* ws,
+                           size_t ws_bytes, cudaStream_t select_stream, cudaStream_t spec_stream,
+                           const prr_step_events* events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRR_H */

@@ -6,11 +6,12 @@
  * (the CUDA library under dynamic_sparse_attention_block_b200/csrc) never calls it,
  * and this file shares no code, header, table or helper with that path.
  *
- * What it computes.  The PRR pages ("Predict, Reuse, and Repair: Accelerating
- * Dynamic Sparse Attention for Long-Context LLM Decoding": abstract; method summary;
- * contribution (3); key result "full top-K coverage without accuracy loss") state
- * that PRR is correctness preserving: its output is exactly that of plain top-K
- * dynamic sparse attention.  So the oracle is that plain definition, per decode step
+ * What it computes.  The PRR pages (Predict, Reuse, and Repair: Accelerating
+ * Dynamic Sparse Attention for Long-Context LLM Decoding -- abstract, method summary,
+ * contribution (3) and the key-result bullet on the repair kernel) state that PRR
+ * preserves correctness: repairing the missed blocks restores full top-K coverage,
+ * so its output is exactly that of plain top-K dynamic sparse attention.  So the
+ * oracle is that plain definition, per decode step
  * and per (sequence b, KV head):
  *   1. per-block key summary: per-channel min and max of the keys of the block
  *      (tokens < n);
@@ -21,7 +22,7 @@
  *   3. true selected set S = the first min(K, nb) blocks under (score desc, index asc);
  *   4. out_h = softmax attention of q_h over exactly the tokens of the blocks in S,
  *      with scale 1/sqrt(d); lse_h = ln sum_i exp(scale*q_h.k_i);
- *   5. EMA predictor (abstract: "lightweight EMA-based predictor"):
+ *   5. EMA predictor (PRR abstract: an exponential moving average of past selections):
  *      e_b <- alpha*e_b + (1-alpha)*[b in S], evaluated as alpha*e + beta*ind with
  *      beta = 1 - alpha, no fused multiply-add (build flag -ffp-contract=off);
  *      Pred_{t+1} = first min(P, nb) blocks under (e desc, index asc).

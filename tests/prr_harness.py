@@ -1,0 +1,136 @@
+"""Drive the CUDA decode path and the fp64 oracle over the same seeded workload and
+compare them.  Inputs come only from ``workloads``; expected values come only from
+``oracle``; nothing computed by the CUDA path is fed to the oracle.
+
+Tolerances (fp32 attention on the GPU against fp64 on the CPU):
+  selected sets, missed sets, keep masks, predicted sets, EMA state: bit-exact;
+  out: max |gpu - oracle| <= 2e-3;  lse: |gpu - oracle| / |oracle| <= 1e-4.
+For Gaussian workloads a differing selected set is accepted when every differing
+block's oracle score lies within 1e-5 * max(1, |s_K|) of the oracle's K-th score
+(the score-gap reading of the repair-sweep workload); such units are then not
+compared on out/lse.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+import oracle as OR
+import workloads as W
+
+OUT_TOL = 2e-3
+LSE_RTOL = 1e-4
+GAP_RTOL = 1e-5
+
+
+def f64(bits):
+    return W.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+@dataclass
+class UnitOracle:
+    """Oracle trajectory of one (sequence, KV head), driven step by step."""
+    w: W.Workload
+    b: int
+    kvh: int
+    k: np.ndarray      # [N0+steps][d] bits
+    v: np.ndarray
+    smin: np.ndarray
+    smax: np.ndarray
+    ema: np.ndarray
+    pred: np.ndarray   # Pred_t (ascending)
+    o: OR.Oracle
+
+    @classmethod
+    def create(cls, w: W.Workload, b: int, kvh: int, steps: int, o: OR.Oracle):
+        k0, v0 = W.kv_prefix(w, b, kvh)
+        kn, vn = W.kv_appended(w, b, kvh, steps)
+        k = np.concatenate([k0, kn])
+        v = np.concatenate([v0, vn])
+        maxnb = w.nb(w.N0 + steps)
+        smin = np.zeros((maxnb, w.d))
+        smax = np.zeros((maxnb, w.d))
+        lo, hi = o.build_summaries(k, w.N0, w.bs)
+        smin[:lo.shape[0]], smax[:lo.shape[0]] = lo, hi
+        ema = np.zeros(maxnb)
+        pred = o.top_ranked(np.zeros(w.nb(w.N0)), w.P) if w.P > 0 else np.zeros(0, np.int32)
+        return cls(w, b, kvh, k, v, smin, smax, ema, pred, o)
+
+    def select(self, t: int, q_bits: np.ndarray):
+        """Summary update for token N0+t, scores, true top-K (all from the oracle)."""
+        w, o = self.w, self.o
+        n = w.N0 + t + 1
+        nb = w.nb(n)
+        tail = (n - 1) // w.bs
+        lo, hi = o.block_summary(self.k, n, w.bs, tail)
+        self.smin[tail], self.smax[tail] = lo, hi
+        qg = f64(q_bits[self.b, self.kvh * w.G:(self.kvh + 1) * w.G])
+        s = o.block_scores(qg, self.smin[:nb], self.smax[:nb])
+        sel = o.top_ranked(s, w.K)
+        return n, nb, qg, s, sel
+
+    def finish(self, n, nb, qg, sel, pred):
+        """Given S_t and the Pred_t actually used: missed/keep, attention, EMA update."""
+        w, o = self.w, self.o
+        missed, keep = o.missed_keep(sel, pred)
+        outs, lses = [], []
+        for g in range(w.G):
+            out, lse = o.attend_blocks(qg[g], self.k, self.v, n, w.bs, sel, w.scale())
+            outs.append(out)
+            lses.append(lse)
+        self.ema[:] = o.ema_update(self.ema, nb, sel, w.alpha)
+        pred_next = o.top_ranked(self.ema[:nb], w.P) if w.P > 0 else np.zeros(0, np.int32)
+        return dict(sel=sel, missed=missed, keep=keep, out=np.stack(outs), lse=np.array(lses),
+                    pred_next=pred_next)
+
+
+def pad(x: Sequence[int], L: int) -> np.ndarray:
+    a = np.full(L, -1, np.int32)
+    a[:len(x)] = x
+    return a
+
+
+@dataclass
+class Report:
+    max_out_err: float = 0.0
+    max_lse_rel: float = 0.0
+    units_compared: int = 0
+    near_tie_units: int = 0
+    messages: List[str] = field(default_factory=list)
+
+    def fail(self, msg: str):
+        self.messages.append(msg)
+
+
+def check_selection(rep: Report, tag: str, gpu_sel: np.ndarray, o_sel: np.ndarray,
+                    scores: np.ndarray, K: int, gaussian: bool) -> bool:
+    """Returns True if sets are identical; records a failure unless a near tie allows it."""
+    g = [int(x) for x in gpu_sel if x >= 0]
+    r = [int(x) for x in o_sel]
+    if g == r:
+        return True
+    if gaussian and len(g) == len(r):
+        kth = np.sort(scores)[::-1][len(r) - 1]
+        tol = GAP_RTOL * max(1.0, abs(kth))
+        diff = set(g) ^ set(r)
+        if all(abs(scores[b] - kth) <= tol for b in diff):
+            rep.near_tie_units += 1
+            return False
+    rep.fail(f"{tag}: selected set differs: gpu={g} oracle={r}")
+    return False
+
+
+def compare_attention(rep: Report, tag: str, gpu_out: np.ndarray, gpu_lse: np.ndarray,
+                      o_out: np.ndarray, o_lse: np.ndarray) -> None:
+    err = float(np.max(np.abs(gpu_out.astype(np.float64) - o_out)))
+    rel = float(np.max(np.abs(gpu_lse.astype(np.float64) - o_lse) / np.maximum(np.abs(o_lse), 1e-30)))
+    rep.max_out_err = max(rep.max_out_err, err)
+    rep.max_lse_rel = max(rep.max_lse_rel, rel)
+    rep.units_compared += 1
+    if not (err <= OUT_TOL) or not math.isfinite(err):
+        rep.fail(f"{tag}: out max-abs error {err:.3e} > {OUT_TOL}")
+    if not (rel <= LSE_RTOL) or not math.isfinite(rel):
+        rep.fail(f"{tag}: lse relative error {rel:.3e} > {LSE_RTOL}")
