@@ -1,0 +1,537 @@
+#!/usr/bin/env python
+"""Benchmark of the PRR decode step (select + speculate + repair): one JSON line.
+
+Metric: microseconds per decode step and KV-tokens/s (B * n per step, the context
+served), with the fraction of the HBM roofline.  Default workload: the
+Llama-3.1-8B-shaped 32K layer (B=1, 32 query / 8 KV heads, d 128, 64-token blocks,
+top-64, budget 64).  Inputs are seeded synthetic data (workloads/).
+
+Timing: W warm-up steps, then exactly K steps, each a CUDA-graph replay of the whole
+step bracketed by CUDA events on the replay stream; the 256 MB L2 flush and the next
+token's KV append run between steps, outside the events.  Per-kernel durations come
+from timing events recorded inside the graph on the kernels' own streams.
+
+Under torchrun (N > 1) every rank runs an independent replica on its own sequences
+(weak scaling, no collective on the data path); value = tokens of all ranks / the max
+over ranks of the summed step time.
+
+--impl reference times the fp64 CPU oracle on the host cores on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "µs/decode step & KV-tokens/s (select+speculate+repair), % of 8 TB/s HBM roofline"
+UNIT = "KV-tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def rank_workload(w: W.Workload, rank: int) -> W.Workload:
+    return w if rank == 0 else w.with_(seed=w.seed + 7919 * rank)
+
+
+def host_cache(w: W.Workload, cap: int):
+    kc = np.zeros((w.B, w.Hkv, cap, w.d), np.uint16)
+    vc = np.zeros_like(kc)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            k0, v0 = W.kv_prefix(w, b, h)
+            kc[b, h, :w.N0], vc[b, h, :w.N0] = k0, v0
+    return kc, vc
+
+
+def appended(w: W.Workload, steps: int):
+    kn = np.empty((steps, w.B, w.Hkv, w.d), np.uint16)
+    vn = np.empty_like(kn)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            k, v = W.kv_appended(w, b, h, steps)
+            kn[:, b, h], vn[:, b, h] = k, v
+    return kn, vn
+
+
+def algorithmic_bytes(w: W.Workload, n: int) -> dict:
+    """Bytes a step must move: all block summaries + K and V of the true top-K blocks."""
+    nb = w.nb(n)
+    keff = min(w.K, nb)
+    summ = w.units * nb * 4 * w.d
+    kv = w.units * keff * w.bs * w.d * 2 * 2  # tail block counted whole (upper bound)
+    return {"summaries": summ, "kv": kv, "total": summ + kv}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, period_ms: int = 50):
+        self.lines = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(period_ms), "-i", gpu_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def wait_first(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.01)
+
+    def stop(self) -> dict:
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names[1:], parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def elapsed_ms(a, b) -> float:
+    """cuEventElapsedTime on two events recorded by the library through their raw
+    handles (torch's own elapsed_time only accepts events torch itself recorded)."""
+    from cuda.bindings import driver
+    err, ms = driver.cuEventElapsedTime(driver.CUevent(init_value=a.cuda_event),
+                                        driver.CUevent(init_value=b.cuda_event))
+    if err != driver.CUresult.CUDA_SUCCESS:
+        raise RuntimeError(f"cuEventElapsedTime: {err}")
+    return float(ms)
+
+
+def kernel_spans(marks) -> dict:
+    """Per-kernel device durations (ms) of the last step from its timing marks."""
+    return {
+        "select": elapsed_ms(marks["t_begin"], marks["t_select_end"]),
+        "repair": elapsed_ms(marks["t_select_end"], marks["t_repair_end"]),
+        "combine": elapsed_ms(marks["t_combine_begin"], marks["t_combine_end"]),
+        "spec": elapsed_ms(marks["t_spec_begin"], marks["t_spec_end"]),
+        "ema": elapsed_ms(marks["t_ema_begin"], marks["t_ema_end"]),
+    }
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dynamic_sparse_attention_block_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken
+    on the current kernel sources (profiles/traffic.txt: kernel workload sha bytes)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = kernel_source_sha()
+    with open(p) as fh:
+        for ln in fh:
+            parts = ln.split()
+            if len(parts) >= 4 and not ln.startswith("#") and parts[0] == kernel \
+                    and parts[1] == workload and parts[2] == sha:
+                return float(parts[3])
+    return None
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+def oracle_run(w: W.Workload, warmup: int, steps: int, budget_s: float, nthreads: int):
+    """Time the fp64 oracle's decode step on the host.  Returns (tokens/s, seconds per
+    step, steps timed, units per step, threads).  Each step runs every (sequence, KV
+    head) unit; the number of timed steps is cut so the loop stays within budget_s."""
+    import oracle as OR
+    o = OR.default()
+    total = warmup + steps
+    cap = w.N0 + total
+    kc, vc = host_cache(w, cap)
+    kn, vn = appended(w, total)
+    qs = W.queries(w, total)
+    st = OR.new_state(w.B, w.Hkv, cap, w.bs, w.d)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            lo, hi = o.build_summaries(kc[b, h], w.N0, w.bs)
+            st["smin"][b, h, :lo.shape[0]], st["smax"][b, h, :lo.shape[0]] = lo, hi
+    dims = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, bs=w.bs, cap=cap, K=w.K, P=w.P, alpha=w.alpha,
+                scale=w.scale())
+    pred = np.full((w.B, w.Hkv, max(w.P, 1)), -1, np.int32)
+    pred[:, :, :min(w.P, w.nb(w.N0))] = np.arange(min(w.P, w.nb(w.N0)))
+    times, tokens, used = [], 0, 1
+    t_start = time.perf_counter()
+    for t in range(total):
+        n = w.N0 + t + 1
+        kc[:, :, n - 1], vc[:, :, n - 1] = kn[t], vn[t]
+        seq = np.full(w.B, n, np.int32)
+        t0 = time.perf_counter()
+        r = o.decode_step(dims, qs[t], kc, vc, seq, pred, st, nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        used = r["threads"]
+        pred = r["pred_next"]
+        if t >= warmup:
+            times.append(dt)
+            tokens += w.B * n
+        if t >= warmup and time.perf_counter() - t_start > budget_s:
+            break
+    secs = sum(times)
+    return tokens / secs, secs / max(len(times), 1), len(times), w.units, used
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = W.workload(args.workload)
+    threads = os.cpu_count() or 1
+    value, sps, nsteps, units, used = oracle_run(w, args.warmup, args.steps, args.ref_budget_s, threads)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": nsteps, "warmup": args.warmup, "ms_per_step": sps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                         "sample": f"{nsteps} full oracle decode steps ({units} (sequence, KV head) "
+                                   f"units each) of {w.name}, OpenMP over units"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    if nsteps < args.steps:
+        line["note"] = f"timed {nsteps} of {args.steps} requested steps (time budget {args.ref_budget_s}s)"
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: W.Workload, args) -> dict:
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "context": w.N0,
+            "block": w.bs, "top_k": w.K, "budget_P": w.P, "alpha": w.alpha, "qk": w.qk,
+            "walk_p": w.walk_p, "l2": "256 MB write between timed steps",
+            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from dynamic_sparse_attention_block_b200 import Dims, PRRDecoder, _abi
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = rank_workload(W.workload(args.workload), rank)
+    hbm_peak, peak_kind = measured_peaks()
+
+    # CPU baseline first (rank 0, N = 1 only), before any GPU work
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        value, sps, nsteps, units, used = oracle_run(W.workload(args.workload), 2, args.cpu_max_steps,
+                                                     args.cpu_budget_s, threads)
+        cpu = {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+               "sample": f"{nsteps} oracle decode steps of {w.name} after 2 warm-up steps "
+                         f"({units} units per step, ~{args.cpu_budget_s:.0f} s budget)"}
+
+    e2e_steps = 0 if args.no_e2e else args.steps
+    cmp_steps = 0 if args.no_streams else min(args.steps, 100)
+    total = 2 + args.warmup + args.steps + e2e_steps + 2 * cmp_steps + 8
+    cap = w.N0 + total
+    dims = Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, bs=w.bs, cap_tokens=cap, K=w.K, P=w.P, alpha=w.alpha)
+    dec = PRRDecoder(dims)
+    kc, vc = host_cache(w, w.N0)
+    dec.k_cache[:, :, :w.N0].copy_(torch.from_numpy(kc.view(np.int16)).view(torch.bfloat16))
+    dec.v_cache[:, :, :w.N0].copy_(torch.from_numpy(vc.view(np.int16)).view(torch.bfloat16))
+    del kc, vc
+    torch.cuda.synchronize()
+    dec.prefill(dec.k_cache[:, :, :w.N0], dec.v_cache[:, :, :w.N0], w.N0)
+    kn, vn = appended(w, total)
+    qs = W.queries(w, total)
+    kn_d = torch.from_numpy(kn.view(np.int16)).cuda().view(torch.bfloat16)
+    vn_d = torch.from_numpy(vn.view(np.int16)).cuda().view(torch.bfloat16)
+    qs_d = torch.from_numpy(qs.view(np.int16)).cuda().view(torch.bfloat16)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    main = torch.cuda.current_stream()
+    marks = {nm: torch.cuda.Event(enable_timing=True) for nm in _abi.TIMING_MARKS}
+    for ev in marks.values():  # torch creates the CUDA event on its first record
+        ev.record(main)
+    t = 0
+
+    def prepare(step):
+        dec.append(kn_d[step], vn_d[step], stream=main)
+        dec.q.copy_(qs_d[step])
+        flush.zero_()
+
+    # eager warm-up of both implementations, then one graph per parity of each
+    for fused in (True, False):
+        prepare(t)
+        main.synchronize()
+        if fused:
+            dec.step_fused(stream=main)
+        else:
+            dec.step(timing=marks)
+        torch.cuda.synchronize()
+        t += 1
+    graphs = {}
+    saved = (dec.parity, dec.fused_parity)
+    for par in (0, 1):
+        dec.parity = par
+        for cpar in (0, 1):  # control-word copy of the fused launch
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=dec.select_stream):
+                dec.step_fused(swap=False, parity=cpar)
+            graphs[("fused", par, cpar)] = g
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=dec.select_stream):
+            dec.step(timing=marks, swap=False)
+        graphs[("streams", par)] = g
+    dec.parity, dec.fused_parity = saved
+    torch.cuda.synchronize()
+
+    def replay(kind):
+        if kind == "fused":
+            graphs[("fused", dec.parity, dec.fused_parity)].replay()
+            dec.fused_parity ^= 1  # consecutive fused launches alternate their control words
+        else:
+            graphs[("streams", dec.parity)].replay()
+        if dims.P > 0:
+            dec.parity ^= 1
+
+    for _ in range(args.warmup):
+        prepare(t)
+        replay("fused")
+        t += 1
+    torch.cuda.synchronize()
+
+    # ---------------- timed region: fused single-launch step
+    clocks = ClockSampler(f"GPU-{torch.cuda.get_device_properties(local).uuid}")
+    clocks.wait_first()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    keep_sum = torch.zeros((), dtype=torch.int64, device="cuda")
+    missed_sum = torch.zeros((), dtype=torch.int64, device="cuda")
+    tokens = 0
+    step_bytes, timed_n = [], []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        prepare(t)
+        starts[i].record(main)
+        replay("fused")
+        ends[i].record(main)
+        keep_sum += dec.keep.sum()
+        missed_sum += dec.n_missed.sum()
+        n = w.N0 + t + 1
+        timed_n.append(n)
+        tokens += w.B * n
+        step_bytes.append(algorithmic_bytes(w, n))
+        t += 1
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    my_time = sum(step_ms) / 1e3
+    status = dec.device_status()
+
+    # ---------------- two-stream implementation on the same trajectory (per-kernel marks)
+    streams = None
+    if cmp_steps:
+        kern = {"select": [], "repair": [], "combine": [], "ema": [], "spec": []}
+        s_ms, overlap_frac = [], []
+        sa = torch.cuda.Event(enable_timing=True)
+        sb = torch.cuda.Event(enable_timing=True)
+        for _ in range(cmp_steps):
+            prepare(t)
+            sa.record(main)
+            replay("streams")
+            sb.record(main)
+            main.synchronize()
+            s_ms.append(sa.elapsed_time(sb))
+            for name, dur in kernel_spans(marks).items():
+                kern[name].append(dur)
+            a1 = elapsed_ms(marks["t_begin"], marks["t_select_end"])
+            b0 = elapsed_ms(marks["t_begin"], marks["t_spec_begin"])
+            b1 = elapsed_ms(marks["t_begin"], marks["t_spec_end"])
+            if b1 > b0:
+                overlap_frac.append(max(0.0, min(a1, b1) - max(0.0, b0)) / (b1 - b0))
+            t += 1
+        streams = {"us_per_step": statistics.mean(s_ms) * 1e3, "steps": cmp_steps,
+                   "kernels_us": {k: statistics.mean(v) * 1e3 for k, v in kern.items()},
+                   "spec_select_overlap": statistics.mean(overlap_frac) if overlap_frac else None,
+                   "gpu_launches_per_step": 4 + (1 if dims.P > 0 else 0)}
+        status = status or dec.device_status()
+
+    # ---------------- end to end: host buffers through the public API
+    e2e = None
+    if e2e_steps:
+        q_h = torch.from_numpy(qs.view(np.int16)).view(torch.bfloat16).pin_memory()
+        kn_h = torch.from_numpy(kn.view(np.int16)).view(torch.bfloat16).pin_memory()
+        vn_h = torch.from_numpy(vn.view(np.int16)).view(torch.bfloat16).pin_memory()
+        out_h = torch.empty(dec.out.shape, dtype=torch.float32).pin_memory()
+        lse_h = torch.empty(dec.lse.shape, dtype=torch.float32).pin_memory()
+        k_stage = torch.empty_like(kn_d[0])
+        v_stage = torch.empty_like(vn_d[0])
+        e_tokens = 0
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+        for i in range(e2e_steps):
+            flush.zero_()
+            es[i].record(main)
+            dec.q.copy_(q_h[t], non_blocking=True)
+            k_stage.copy_(kn_h[t], non_blocking=True)
+            v_stage.copy_(vn_h[t], non_blocking=True)
+            dec.append(k_stage, v_stage, stream=main)
+            replay("fused")
+            out_h.copy_(dec.out, non_blocking=True)
+            lse_h.copy_(dec.lse, non_blocking=True)
+            ee[i].record(main)
+            main.synchronize()
+            e_tokens += w.B * (w.N0 + t + 1)
+            t += 1
+        e_ms = [a.elapsed_time(b) for a, b in zip(es, ee)]
+        h2d = q_h[0].numel() * 2 + kn_h[0].numel() * 2 * 2
+        d2h = out_h.numel() * 4 + lse_h.numel() * 4
+        e2e = {"value": e_tokens / (sum(e_ms) / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": statistics.mean(e_ms),
+               "path": "append + fused step graph + D2H of out/lse, pinned host buffers"}
+        if not np.all(np.isfinite(out_h.numpy())):
+            status = status or -1
+
+    # ---------------- reduce over ranks
+    tot_tokens, max_time = tokens, my_time
+    if world > 1:
+        tt = torch.tensor([float(tokens)], device="cuda")
+        mt = torch.tensor([my_time], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.SUM)
+        dist.all_reduce(mt, op=dist.ReduceOp.MAX)
+        tot_tokens, max_time = tt.item(), mt.item()
+        if e2e is not None:
+            ev = torch.tensor([e2e["value"]], device="cuda")
+            dist.all_reduce(ev, op=dist.ReduceOp.SUM)
+            e2e["value"] = ev.item()
+    value = tot_tokens / max_time
+
+    # ---------------- roofline: the fused step kernel is the step's only kernel
+    keff = min(w.K, w.nb(w.N0))
+    overlap = keep_sum.item() / (args.steps * w.units * keff) if w.P > 0 else 0.0
+    step_algo = statistics.mean(b["total"] for b in step_bytes)
+    step_mean_ms = statistics.mean(step_ms)
+    achieved = step_algo / (step_mean_ms * 1e-3) / 1e9
+    traffic = recorded_traffic("fused_step_kernel", w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_mean_ms, "us_per_step": step_mean_ms * 1e3,
+        "us_per_step_p50": statistics.median(step_ms) * 1e3,
+        "us_per_step_p90": float(np.percentile(step_ms, 90)) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(w, args),
+        "roofline": {"bound": "hbm", "kernel": "fused_step_kernel", "achieved": achieved, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} copy bandwidth (burst)",
+                     "algorithmic_bytes_per_launch": step_algo, "avg_launch_us": step_mean_ms * 1e3},
+        "step_roofline": {"algorithmic_bytes_per_step": step_algo, "achieved_gbs": achieved,
+                          "frac_of_8tbs": achieved / NOMINAL_HBM_GBS, "frac_of_measured": achieved / hbm_peak},
+        "predictor_overlap": overlap,
+        "repaired_blocks_per_unit": missed_sum.item() / (args.steps * w.units),
+        "streams_path": streams,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+        "clocks": clk, "device_status": status,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs.values():
+        g.reset()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if status == 0 else 1
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("prr", "reference"), default="prr")
+    ap.add_argument("--workload", default="llama8b_32k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-streams", action="store_true", help="skip the two-stream comparison run")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--cpu-max-steps", type=int, default=1500)
+    ap.add_argument("--ref-budget-s", type=float, default=150.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -30,13 +30,16 @@ class PrrDims(ctypes.Structure):
 class PrrStepBuffers(ctypes.Structure):
     _fields_ = [(n, _c_void_p) for n in (
         "q", "k_cache", "v_cache", "seq_lens", "summ", "ema", "pred", "pred_next", "sel",
-        "missed", "n_missed", "keep", "part_m", "part_l", "part_O", "out", "lse")]
+        "missed", "n_missed", "keep", "part_m", "part_l", "part_O", "out", "lse", "trace")]
+
+
+STEP_EVENTS = ("fork", "sel_done", "spec_done", "join")
+TIMING_MARKS = ("t_begin", "t_select_end", "t_repair_end", "t_combine_begin", "t_combine_end",
+                "t_spec_begin", "t_spec_end", "t_ema_begin", "t_ema_end")
 
 
 class PrrStepEvents(ctypes.Structure):
-    _fields_ = [(n, _c_void_p) for n in (
-        "fork", "join", "t_begin", "t_select_end", "t_repair_end", "t_ema_end", "t_spec_begin",
-        "t_spec_end")]
+    _fields_ = [(n, _c_void_p) for n in STEP_EVENTS + TIMING_MARKS]
 
 
 # exported C symbols, in header order
@@ -44,6 +47,7 @@ SYMBOLS = (
     "prr_version", "prr_status_string", "prr_workspace_bytes", "prr_workspace_init",
     "prr_get_device_status", "prr_append_kv", "prr_update_summaries", "prr_select_topk",
     "prr_ema_predict", "prr_speculate", "prr_repair_merge", "prr_decode_step",
+    "prr_decode_step_fused",
 )
 
 STATUS = {0: "PRR_OK", 1: "PRR_ERR_INVALID_ARG", 2: "PRR_ERR_SHAPE", 3: "PRR_ERR_CAPACITY",
@@ -91,6 +95,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     L.prr_repair_merge.argtypes = [dims, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.prr_decode_step.argtypes = [dims, ctypes.POINTER(PrrStepBuffers), vp, sz, vp, vp,
                                   ctypes.POINTER(PrrStepEvents)]
+    L.prr_decode_step_fused.argtypes = [dims, ctypes.POINTER(PrrStepBuffers), vp, sz, _i32, vp]
     for name in SYMBOLS:
         if name not in ("prr_version", "prr_status_string", "prr_workspace_bytes"):
             getattr(L, name).restype = ctypes.c_int
@@ -237,3 +242,10 @@ def prr_decode_step(dims, buffers: PrrStepBuffers, ws, select_stream, spec_strea
                                   ws.numel() * ws.element_size(), _stream(select_stream),
                                   _stream(spec_stream), ctypes.byref(events)),
            "prr_decode_step")
+
+
+def prr_decode_step_fused(dims, buffers: PrrStepBuffers, ws, step_parity: int, stream=None) -> None:
+    _check(load().prr_decode_step_fused(ctypes.byref(_dims(dims)), ctypes.byref(buffers), _ptr(ws),
+                                        ws.numel() * ws.element_size(), int(step_parity),
+                                        _stream(stream)),
+           "prr_decode_step_fused")

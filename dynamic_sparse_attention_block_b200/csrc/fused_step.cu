@@ -1,0 +1,355 @@
+// fused_step.cu -- the whole PRR decode step in ONE persistent launch.
+//
+// Resident CTAs (128 threads) take work items from one atomic counter, in this order:
+//   1. SEL     (unit, chunk of 128 blocks): tail-summary fold, block scores -> keys; the
+//              last chunk of a unit runs the top-K finisher and publishes S_t.
+//   2. SPEC    (unit, predicted slot): speculative partial of block Pred_t[slot].  A
+//              speculative item that starts after its unit's selection is published
+//              skips a block that selection dropped (its partial would be discarded).
+//   3. REPAIR  (unit, missed slot): partial of a missed block (waits for S_t).
+//   4. EMA     (unit): predictor update with S_t and Pred_{t+1} (waits for S_t).
+//   5. COMBINE (unit, query head): LSE merge of kept + repaired partials (waits for all
+//              of the unit's speculative and repair partials).
+// This is the PRR runtime (abstract; method summary; contributions (1)-(3)) scheduled
+// for a 148-SM part: speculation overlaps selection inside the launch, selection work
+// is handed out first so the critical path (select -> repair -> merge) starts at once,
+// and no kernel boundary separates the phases.
+//
+// Waits only ever target items with a smaller index, which were taken by CTAs that are
+// already running, so every wait ends without any co-residency assumption.  Each wait
+// is bounded (kWaitLimitNs); a timeout records kDevWaitTimeout and raises an abort flag
+// that makes every later wait give up at once.
+//
+// Control words live in the workspace in two copies selected by the step parity: a
+// launch works on copy[parity] and clears copy[1 - parity] for the next launch, so no
+// reset launch is needed and a late CTA can never see the next step's counters.
+#include "prr_attn.cuh"
+#include "prr_parts.cuh"
+
+namespace prr {
+
+constexpr int kFusedChunk = 128;  // blocks per SEL item (4 warps x 32 rows)
+
+struct FusedCtl {
+  unsigned* work;      // next item
+  unsigned* abort;     // set on a timed-out wait
+  unsigned* sel_cnt;   // [units] finished SEL chunks
+  unsigned* sel_done;  // [units] S_t published
+  unsigned* target;    // [units] active speculative slots + missed blocks
+  unsigned* done_cnt;  // [units] finished speculative + repair items
+};
+
+__device__ __forceinline__ FusedCtl ctl_view(const Params& p, int parity) {
+  unsigned* b = p.ctl + static_cast<size_t>(parity) * p.ctl_words;
+  const int U = p.units;
+  return FusedCtl{b, b + 1, b + 16, b + 16 + U, b + 16 + 2 * U, b + 16 + 3 * U};
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// CTA-wide bounded wait until *flag >= target.  Thread 0 polls; the verdict is shared.
+__device__ bool wait_geq(const unsigned* flag, unsigned target, const FusedCtl& C, int* status, int* sh) {
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    if (ld_acquire(flag) < target) {
+      const uint64_t t0 = global_ns();
+      for (;;) {
+        if (ld_acquire(flag) >= target) break;
+        if (ld_acquire(C.abort)) {
+          ok = 0;
+          break;
+        }
+        if (global_ns() - t0 > kWaitLimitNs) {
+          report(status, kDevWaitTimeout);
+          atomicExch(C.abort, 1u);
+          ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    sh[0] = ok;
+  }
+  __syncthreads();
+  const bool ok = sh[0] != 0;
+  __syncthreads();
+  return ok;
+}
+
+__device__ __forceinline__ void count_done(unsigned* counter) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) atomicAdd(counter, 1u);
+}
+
+template <int D>
+struct FusedSel {
+  static constexpr int ROWB = 4 * D;
+  static constexpr int C = ROWB / 16;
+  __host__ __device__ static size_t aux(int maxnb) {  // coefficient area follows tiles / finisher scratch
+    size_t a = static_cast<size_t>(kFusedChunk) * ROWB;
+    const size_t f = finish_scratch_bytes(maxnb);
+    if (f > a) a = f;
+    return (a + 15) & ~static_cast<size_t>(15);
+  }
+  __host__ __device__ static size_t bytes(int maxnb) { return aux(maxnb) + 2 * C * 16 + 2 * D; }
+};
+
+// ---------------------------------------------------------------- SEL item
+template <int D>
+__device__ void sel_item(const Params& p, const FusedCtl& C, int u, int chunk, unsigned char* smem, uint64_t* bar,
+                         uint32_t& ph, int* sh) {
+  using L = FusedSel<D>;
+  constexpr int ROWB = L::ROWB;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = checked_len(p, u / p.Hkv);
+  const int nb = (n + p.bs - 1) / p.bs;
+  const int c0 = chunk * kFusedChunk;
+  const int cnt = max(0, min(kFusedChunk, nb - c0));
+  const int tail = n > 0 ? (n - 1) / p.bs : -1;
+  const bool own_tail = p.append_summary && tail >= c0 && tail < c0 + cnt;
+  uint16_t* summ_unit = p.summ + static_cast<size_t>(u) * p.maxnb * 2 * D;
+  const size_t aux = L::aux(p.maxnb);
+  float4* coef_lo = reinterpret_cast<float4*>(smem + aux);
+  float4* coef_hi = coef_lo + L::C;
+  uint16_t* newk = reinterpret_cast<uint16_t*>(coef_hi + L::C);
+
+  if (tid == 0 && cnt > 0) {
+    fence_proxy_async();
+    mbar_expect_tx(bar, static_cast<uint32_t>(cnt) * ROWB);
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(summ_unit) + static_cast<size_t>(c0) * ROWB;
+    for (int w = 0; w < 4; ++w) {
+      const int rows = min(32, cnt - 32 * w);
+      if (rows > 0) bulk_load(smem + w * 32 * ROWB, src + static_cast<size_t>(w) * 32 * ROWB, rows * ROWB, bar);
+    }
+  }
+  load_group_coef<D>(p, u, coef_lo, coef_hi);
+  if (own_tail) {
+    const uint16_t* krow = p.kc + (static_cast<size_t>(u) * p.cap + (n - 1)) * D;
+    for (int c = tid; c < D / 8; c += blockDim.x)
+      reinterpret_cast<uint4*>(newk)[c] = __ldg(reinterpret_cast<const uint4*>(krow) + c);
+  }
+  __syncthreads();
+  if (cnt > 0) {
+    const bool ok = __syncthreads_and(mbar_wait(bar, ph, p.status));
+    ph ^= 1u;
+    if (!ok) {
+      if (tid == 0) atomicExch(C.abort, 1u);
+      return;
+    }
+  }
+  const int first = c0 + 32 * warp;
+  const int rows = min(32, cnt - 32 * warp);
+  if (rows > 0) {
+    unsigned char* tile = smem + warp * 32 * ROWB;
+    if (own_tail && tail >= first && tail < first + rows)
+      fold_tail_row<D>(reinterpret_cast<uint32_t*>(tile + (tail - first) * ROWB), newk, ((n - 1) % p.bs) == 0,
+                       reinterpret_cast<uint32_t*>(summ_unit + static_cast<size_t>(tail) * 2 * D), lane);
+    if (lane < rows)
+      p.keys[static_cast<size_t>(u) * p.maxnb + first + lane] =
+          orderable(score_summary_row<D>(tile + lane * ROWB, coef_lo, coef_hi, lane));
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sh[1] = (atomicAdd(C.sel_cnt + u, 1u) == static_cast<unsigned>(p.fchunks - 1)) ? 1 : 0;
+  __syncthreads();
+  if (!sh[1]) return;
+  __threadfence();
+  const FinishOut f = select_finish(p, u, nb, smem);  // tiles are dead: scratch at 0
+  __threadfence();  // every thread's outputs are visible before S_t is published
+  __syncthreads();
+  if (tid == 0) {
+    C.target[u] = static_cast<unsigned>(f.p_active + f.n_missed);
+    __threadfence();
+    atomicExch(C.sel_done + u, 1u);
+  }
+}
+
+// ---------------------------------------------------------------- fused kernel
+template <int D, int BS>
+__global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                         const __grid_constant__ CUtensorMap vmap,
+                                                         const __grid_constant__ Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.fused_region);  // K tile, V tile, summaries
+  int* sh = reinterpret_cast<int*>(bars + 3);                              // broadcast slots
+  const int tid = threadIdx.x;
+  const FusedCtl C = ctl_view(p, p.parity);
+
+  if (blockIdx.x == 0) {  // clear the other copy of the control words for the next launch
+    unsigned* other = p.ctl + static_cast<size_t>(1 - p.parity) * p.ctl_words;
+    for (int i = tid; i < p.ctl_words; i += blockDim.x) other[i] = 0u;
+  }
+  if (tid == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  uint32_t ph_attn = 0u, ph_sel = 0u;
+  const int U = p.units;
+  const int n_sel = U * p.fchunks, n_spec = U * p.P, n_rep = U * p.K, n_ema = U;
+  const int n_comb = U * p.G;
+  const int total = n_sel + n_spec + n_rep + n_ema + n_comb;
+
+  for (;;) {
+    if (tid == 0) sh[2] = static_cast<int>(atomicAdd(C.work, 1u));
+    __syncthreads();
+    int it = sh[2];
+    __syncthreads();
+    if (it >= total) break;
+    fence_proxy_async();  // generic shared-memory writes of the last item precede new copies
+    if (p.trace && tid == 0) {
+      unsigned smid;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+      p.trace[4 * static_cast<size_t>(it) + 0] = global_ns();
+      p.trace[4 * static_cast<size_t>(it) + 2] = (static_cast<unsigned long long>(smid) << 32) | blockIdx.x;
+      p.trace[4 * static_cast<size_t>(it) + 3] = static_cast<unsigned long long>(it);
+    }
+    const int item_id = it;
+
+    if (it < n_sel) {
+      sel_item<D>(p, C, it / p.fchunks, it % p.fchunks, smem, &bars[2], ph_sel, sh);
+      __syncthreads();
+      if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
+      continue;
+    }
+    it -= n_sel;
+    if (it < n_spec) {  // speculation
+      const int u = it / p.P, j = it % p.P;
+      const int n = checked_len(p, u / p.Hkv);
+      const int nb = (n + BS - 1) / BS;
+      const int blk = p.pred[static_cast<size_t>(u) * p.P + j];
+      if (blk >= 0 && blk < nb) {
+        if (tid == 0) sh[3] = (ld_acquire(C.sel_done + u) != 0u &&
+                               __ldcg(p.keep + static_cast<size_t>(u) * p.P + j) == 0) ? 1 : 0;
+        __syncthreads();
+        const bool skip = sh[3] != 0;
+        if (!skip) {
+          const size_t row0 = static_cast<size_t>(u) * p.G * p.P + j;
+          const PartialDst dst{p.pm + row0, p.pl + row0, p.pO + row0 * D, static_cast<size_t>(p.P),
+                               static_cast<size_t>(p.P) * D};
+          if (!block_partial<D, BS>(p, &kmap, &vmap, u, blk, n, dst, smem, bars, ph_attn) && tid == 0)
+            atomicExch(C.abort, 1u);
+          ph_attn ^= 1u;
+        }
+        count_done(C.done_cnt + u);
+      }
+      __syncthreads();
+      if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
+      continue;
+    }
+    it -= n_spec;
+    if (it < n_rep) {  // repair
+      const int u = it / p.K, i = it % p.K;
+      if (wait_geq(C.sel_done + u, 1u, C, p.status, sh)) {
+        const int nm = min(max(__ldcg(p.n_missed + u), 0), p.K);
+        if (i < nm) {
+          const int n = checked_len(p, u / p.Hkv);
+          const int nb = (n + BS - 1) / BS;
+          const int blk = __ldcg(p.missed + static_cast<size_t>(u) * p.K + i);
+          const size_t row0 = static_cast<size_t>(u) * p.G * p.K + i;
+          const PartialDst dst{p.rm + row0, p.rl + row0, p.rO + row0 * D, static_cast<size_t>(p.K),
+                               static_cast<size_t>(p.K) * D};
+          if (blk >= 0 && blk < nb) {
+            if (!block_partial<D, BS>(p, &kmap, &vmap, u, blk, n, dst, smem, bars, ph_attn) && tid == 0)
+              atomicExch(C.abort, 1u);
+            ph_attn ^= 1u;
+          } else {
+            if (tid == 0) report(p.status, kDevBadMissed);
+            write_empty_partial(dst, p.G, D);
+          }
+          count_done(C.done_cnt + u);
+        }
+      }
+      __syncthreads();
+      if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
+      continue;
+    }
+    it -= n_rep;
+    if (it < n_ema) {  // predictor for step t+1
+      if (wait_geq(C.sel_done + it, 1u, C, p.status, sh)) ema_unit(p, it, smem);
+      __syncthreads();
+      if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
+      continue;
+    }
+    it -= n_ema;
+    {  // LSE merge of (unit, head)
+      const int u = it / p.G, h = it % p.G;
+      if (wait_geq(C.sel_done + u, 1u, C, p.status, sh)) {
+        const unsigned tgt = __ldcg(C.target + u);
+        if (wait_geq(C.done_cnt + u, tgt, C, p.status, sh)) combine_head<D>(p, u, h, smem);
+      }
+      __syncthreads();
+      if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
+    }
+  }
+}
+
+template <int D, int BS>
+static size_t fused_region_bytes(const Params& p) {
+  size_t r = FusedSel<D>::bytes(p.maxnb);
+  r = r > AttnTile<D, BS>::bytes ? r : AttnTile<D, BS>::bytes;
+  const size_t e = ema_scratch_bytes(p.maxnb);
+  r = r > e ? r : e;
+  const size_t c = combine_scratch_bytes(p.P, p.K, D);
+  r = r > c ? r : c;
+  return (r + 15) & ~static_cast<size_t>(15);
+}
+
+template <int D, int BS>
+static cudaError_t launch_fused_t(Params p, const CUtensorMap& kmap, const CUtensorMap& vmap, cudaStream_t s,
+                                  int priority, int sms, int* grid_out) {
+  p.fchunks = (p.maxnb + kFusedChunk - 1) / kFusedChunk;
+  p.fused_region = static_cast<int>(fused_region_bytes<D, BS>(p));
+  const size_t smem = 1024 + static_cast<size_t>(p.fused_region) + 3 * 8 + 8 * 4;
+  const void* fn = reinterpret_cast<const void*>(fused_step_kernel<D, BS>);
+  cudaError_t e = allow_max_smem(fn);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_step_kernel<D, BS>, 128, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const long long items = static_cast<long long>(p.units) * (p.fchunks + p.P + p.K + 1 + p.G);
+  long long grid = static_cast<long long>(per_sm) * sms;
+  if (grid > items) grid = items;
+  if (grid_out) *grid_out = static_cast<int>(grid);
+  return launch_kernel(fused_step_kernel<D, BS>, dim3(static_cast<unsigned>(grid)), dim3(128), smem, s, priority,
+                       kmap, vmap, p);
+}
+
+cudaError_t launch_fused(const Params& p, const CUtensorMap& kmap, const CUtensorMap& vmap, cudaStream_t s,
+                         int priority, int sms, int* grid_out) {
+  if (p.d == 128) {
+    if (p.bs == 128) return launch_fused_t<128, 128>(p, kmap, vmap, s, priority, sms, grid_out);
+    return launch_fused_t<128, 64>(p, kmap, vmap, s, priority, sms, grid_out);
+  }
+  if (p.bs == 128) return launch_fused_t<64, 128>(p, kmap, vmap, s, priority, sms, grid_out);
+  return launch_fused_t<64, 64>(p, kmap, vmap, s, priority, sms, grid_out);
+}
+
+size_t fused_smem_bytes(const Params& p) {
+  Params q = p;
+  q.fchunks = (q.maxnb + kFusedChunk - 1) / kFusedChunk;
+  size_t r;
+  if (p.d == 128) r = p.bs == 128 ? fused_region_bytes<128, 128>(q) : fused_region_bytes<128, 64>(q);
+  else r = p.bs == 128 ? fused_region_bytes<64, 128>(q) : fused_region_bytes<64, 64>(q);
+  return 1024 + r + 3 * 8 + 8 * 4;
+}
+
+}  // namespace prr
+
+#ifdef PRR_PHASE_DEBUG
+// Debug builds only: copy the phase timestamps of the fused kernel's translation unit.
+extern "C" int prr_debug_phases(void* dst) {
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, prr::g_phase, sizeof(prr::g_phase)));
+}
+#endif

@@ -21,8 +21,6 @@ constexpr int kVersion = 100;  // 0.1.0
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-int list_len_for(int K) { return K <= 32 ? 32 : (K <= 64 ? 64 : 128); }
-
 bool dims_ok(const prr_dims* d) {
   if (!d) return false;
   if (d->B < 1 || d->Hkv < 1 || d->Hq < d->Hkv || d->Hq % d->Hkv) return false;
@@ -40,26 +38,24 @@ bool dims_ok(const prr_dims* d) {
 
 WsLayout layout_for(const prr_dims* d) {
   WsLayout L = {};
-  const int units = d->B * d->Hkv;
-  const int G = d->Hq / d->Hkv;
-  const int maxnb = (d->cap_tokens + d->bs - 1) / d->bs;
-  L.list_len = list_len_for(d->K);
-  L.max_chunks = (maxnb + 31) / 32;
+  const size_t units = static_cast<size_t>(d->B) * d->Hkv;
+  const size_t G = static_cast<size_t>(d->Hq / d->Hkv);
+  const size_t maxnb = static_cast<size_t>((d->cap_tokens + d->bs - 1) / d->bs);
   size_t off = 0;
   L.status = off;
   off = align256(off + 4);
   L.sel_cnt = off;
-  off = align256(off + 4 * static_cast<size_t>(units));
-  L.merge_cnt = off;
-  off = align256(off + 4 * static_cast<size_t>(units));
-  L.cand = off;
-  off = align256(off + 8 * static_cast<size_t>(units) * L.max_chunks * L.list_len);
+  off = align256(off + 4 * units);
+  L.keys = off;
+  off = align256(off + 4 * units * maxnb);
   L.rm = off;
-  off = align256(off + 4 * static_cast<size_t>(units) * G * d->K);
+  off = align256(off + 4 * units * G * d->K);
   L.rl = off;
-  off = align256(off + 4 * static_cast<size_t>(units) * G * d->K);
+  off = align256(off + 4 * units * G * d->K);
   L.rO = off;
-  off = align256(off + 4 * static_cast<size_t>(units) * G * d->K * d->d);
+  off = align256(off + 4 * units * G * d->K * d->d);
+  L.ctl = off;
+  off = align256(off + 4 * 2 * (16 + 4 * units));
   L.total = off;
   return L;
 }
@@ -107,7 +103,7 @@ int select_chunk(int units, int maxnb, int sms) {
   return static_cast<int>(c);
 }
 
-Params base_params(const prr_dims* d, void* ws, int mode) {
+Params base_params(const prr_dims* d, void* ws) {
   Params p;
   std::memset(&p, 0, sizeof p);
   p.B = d->B;
@@ -123,22 +119,31 @@ Params base_params(const prr_dims* d, void* ws, int mode) {
   p.units = d->B * d->Hkv;
   p.scale_log2 = static_cast<float>(static_cast<double>(d->scale) * 1.4426950408889634074);
   p.alpha = d->alpha;
-  p.mode = mode;
-  const WsLayout L = layout_for(d);
-  p.list_len = L.list_len;
   p.chunk_blocks = select_chunk(p.units, p.maxnb, device_info().sms);
   p.nchunks = (p.maxnb + p.chunk_blocks - 1) / p.chunk_blocks;
+  const WsLayout L = layout_for(d);
   unsigned char* w = static_cast<unsigned char*>(ws);
   if (w) {
     p.status = reinterpret_cast<int*>(w + L.status);
     p.sel_cnt = reinterpret_cast<unsigned*>(w + L.sel_cnt);
-    p.merge_cnt = reinterpret_cast<unsigned*>(w + L.merge_cnt);
-    p.cand = reinterpret_cast<uint64_t*>(w + L.cand);
+    p.keys = reinterpret_cast<uint32_t*>(w + L.keys);
     p.rm = reinterpret_cast<float*>(w + L.rm);
     p.rl = reinterpret_cast<float*>(w + L.rl);
     p.rO = reinterpret_cast<float*>(w + L.rO);
+    p.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
   }
+  p.ctl_words = 16 + 4 * p.units;
   return p;
+}
+
+// Record a timing mark; under stream capture it must become a real event-record node.
+cudaError_t record_mark(cudaEvent_t ev, cudaStream_t s) {
+  if (!ev) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                                             : cudaEventRecord(ev, s);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
@@ -240,7 +245,7 @@ prr_status prr_append_kv(const prr_dims* dims, const uint16_t* k_new, const uint
   if (!k_new || !v_new || !seq_lens || !k_cache || !v_cache || !ws) return PRR_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
     return PRR_ERR_INVALID_ARG;
-  Params p = base_params(dims, ws, MODE_STANDALONE);
+  Params p = base_params(dims, ws);
   return cuda_status(launch_append_kv(p, k_new, v_new, k_cache, v_cache, seq_lens, stream));
 }
 
@@ -255,7 +260,7 @@ prr_status prr_update_summaries(const prr_dims* dims, const uint16_t* k_cache,
   if (!aligned16(k_cache) || !aligned16(summ)) return PRR_ERR_INVALID_ARG;
   if (max_range_tokens < 1 || max_range_tokens > dims->cap_tokens) return PRR_ERR_SHAPE;
   if (!tok_begin && max_range_tokens != 1) return PRR_ERR_SHAPE;
-  Params p = base_params(dims, ws, MODE_STANDALONE);
+  Params p = base_params(dims, ws);
   p.kc = k_cache;
   p.summ = summ;
   p.seq_lens = seq_lens;
@@ -272,7 +277,7 @@ prr_status prr_select_topk(const prr_dims* dims, const uint16_t* q, const uint16
   if (!q || !summ || !seq_lens || !sel || !missed || !n_missed || !ws) return PRR_ERR_INVALID_ARG;
   if (dims->P > 0 && (!pred || !keep)) return PRR_ERR_INVALID_ARG;
   if (!aligned16(summ)) return PRR_ERR_INVALID_ARG;
-  Params p = base_params(dims, ws, MODE_STANDALONE);
+  Params p = base_params(dims, ws);
   p.q = q;
   p.summ = const_cast<uint16_t*>(summ);
   p.seq_lens = seq_lens;
@@ -289,8 +294,7 @@ prr_status prr_ema_predict(const prr_dims* dims, double* ema, const int32_t* sel
                            cudaStream_t stream) {
   if (!dims_ok(dims)) return PRR_ERR_SHAPE;
   if (!ema || !seq_lens || !ws || (dims->P > 0 && !pred_next)) return PRR_ERR_INVALID_ARG;
-  if (dims->P == 0 && !sel) return PRR_OK;
-  Params p = base_params(dims, ws, MODE_STANDALONE);
+  Params p = base_params(dims, ws);
   p.ema = ema;
   p.sel = const_cast<int*>(sel);
   p.seq_lens = seq_lens;
@@ -307,7 +311,7 @@ prr_status prr_speculate(const prr_dims* dims, const uint16_t* q, const uint16_t
   if (!q || !k_cache || !v_cache || !seq_lens || !pred || !part_m || !part_l || !part_O || !ws)
     return PRR_ERR_INVALID_ARG;
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(part_O)) return PRR_ERR_INVALID_ARG;
-  Params p = base_params(dims, ws, MODE_STANDALONE);
+  Params p = base_params(dims, ws);
   p.q = q;
   p.kc = k_cache;
   p.vc = v_cache;
@@ -333,7 +337,7 @@ prr_status prr_repair_merge(const prr_dims* dims, const uint16_t* q, const uint1
   if (dims->P > 0 && (!keep || !pred || !part_m || !part_l || !part_O)) return PRR_ERR_INVALID_ARG;
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PRR_ERR_INVALID_ARG;
   if (part_O && !aligned16(part_O)) return PRR_ERR_INVALID_ARG;
-  Params p = base_params(dims, ws, MODE_STANDALONE);
+  Params p = base_params(dims, ws);
   p.q = q;
   p.kc = k_cache;
   p.vc = v_cache;
@@ -349,14 +353,19 @@ prr_status prr_repair_merge(const prr_dims* dims, const uint16_t* q, const uint1
   p.lse = lse;
   CUtensorMap km, vm;
   if (!make_kv_map(&km, k_cache, dims) || !make_kv_map(&vm, v_cache, dims)) return PRR_ERR_CUDA;
-  return cuda_status(launch_attention(p, km, vm, 1, stream, 0));
+  cudaError_t e = launch_attention(p, km, vm, 1, stream, 0);
+  if (e == cudaSuccess) e = launch_combine(p, stream, 0);
+  return cuda_status(e);
 }
 
-prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* b, void* ws,
-                           size_t ws_bytes, cudaStream_t select_stream, cudaStream_t spec_stream,
-                           const prr_step_events* ev) {
+}  // extern "C"
+
+namespace {
+
+// Shared validation of the step buffers; fills the kernel parameter block.
+prr_status step_params(const prr_dims* dims, const prr_step_buffers* b, void* ws, size_t ws_bytes, Params* out) {
   if (!dims_ok(dims)) return PRR_ERR_SHAPE;
-  if (!b || !ws || !ev || !ev->fork || !ev->join) return PRR_ERR_INVALID_ARG;
+  if (!b || !ws) return PRR_ERR_INVALID_ARG;
   if (ws_bytes < layout_for(dims).total) return PRR_ERR_CAPACITY;
   if (!b->q || !b->k_cache || !b->v_cache || !b->seq_lens || !b->summ || !b->ema || !b->sel ||
       !b->missed || !b->n_missed || !b->out || !b->lse)
@@ -367,8 +376,7 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* b, void
   if (!aligned16(b->k_cache) || !aligned16(b->v_cache) || !aligned16(b->summ) || !aligned16(b->out))
     return PRR_ERR_INVALID_ARG;
   if (b->part_O && !aligned16(b->part_O)) return PRR_ERR_INVALID_ARG;
-
-  Params p = base_params(dims, ws, MODE_STEP);
+  Params p = base_params(dims, ws);
   p.q = b->q;
   p.kc = b->k_cache;
   p.vc = b->v_cache;
@@ -386,44 +394,75 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* b, void
   p.pO = b->part_O;
   p.out = b->out;
   p.lse = b->lse;
+  p.append_summary = 1;
+  p.trace = b->trace;
+  *out = p;
+  return PRR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* b, void* ws,
+                           size_t ws_bytes, cudaStream_t select_stream, cudaStream_t spec_stream,
+                           const prr_step_events* ev) {
+  if (!ev || !ev->fork || !ev->sel_done || !ev->spec_done || !ev->join) return PRR_ERR_INVALID_ARG;
+  Params p;
+  const prr_status st = step_params(dims, b, ws, ws_bytes, &p);
+  if (st != PRR_OK) return st;
   CUtensorMap km, vm;
   if (!make_kv_map(&km, b->k_cache, dims) || !make_kv_map(&vm, b->v_cache, dims)) return PRR_ERR_CUDA;
   const DeviceInfo di = device_info();
   const int hi = di.prio_high, lo = di.prio_low;
 
-  cudaError_t e;
-#define PRR_TRY(x)                         \
-  do {                                     \
-    e = (x);                               \
-    if (e != cudaSuccess) return PRR_ERR_CUDA; \
+#define PRR_TRY(x)                               \
+  do {                                           \
+    if ((x) != cudaSuccess) return PRR_ERR_CUDA; \
   } while (0)
-  PRR_TRY(cudaEventRecord(ev->fork, select_stream));
-  PRR_TRY(cudaStreamWaitEvent(spec_stream, ev->fork, 0));
-  // speculation on Pred_t: independent of selection
-  if (ev->t_spec_begin) PRR_TRY(cudaEventRecord(ev->t_spec_begin, spec_stream));
-  PRR_TRY(launch_attention(p, km, vm, 0, spec_stream, lo));
-  if (ev->t_spec_end) PRR_TRY(cudaEventRecord(ev->t_spec_end, spec_stream));
-  // critical path: tail summary -> selection -> repair
-  if (ev->t_begin) PRR_TRY(cudaEventRecord(ev->t_begin, select_stream));
-  {
-    Params ps = p;
-    ps.tok_begin = nullptr;
-    ps.tok_end = nullptr;
-    PRR_TRY(launch_update_summaries(ps, 1, select_stream, hi));
-  }
-  PRR_TRY(launch_select(p, select_stream, hi));
-  if (ev->t_select_end) PRR_TRY(cudaEventRecord(ev->t_select_end, select_stream));
-  PRR_TRY(launch_attention(p, km, vm, 1, select_stream, hi));
-  if (ev->t_repair_end) PRR_TRY(cudaEventRecord(ev->t_repair_end, select_stream));
-  if (dims->P > 0) {
-    Params pe = p;
-    PRR_TRY(launch_ema(pe, select_stream, lo));
-  }
-  if (ev->t_ema_end) PRR_TRY(cudaEventRecord(ev->t_ema_end, select_stream));
-  PRR_TRY(cudaEventRecord(ev->join, spec_stream));
-  PRR_TRY(cudaStreamWaitEvent(select_stream, ev->join, 0));
+  cudaStream_t A = select_stream, B = spec_stream;
+  PRR_TRY(cudaEventRecord(ev->fork, A));
+  PRR_TRY(cudaStreamWaitEvent(B, ev->fork, 0));
+  // spec stream: speculation over Pred_t, independent of selection
+  PRR_TRY(record_mark(ev->t_spec_begin, B));
+  PRR_TRY(launch_attention(p, km, vm, 0, B, lo));
+  PRR_TRY(record_mark(ev->t_spec_end, B));
+  PRR_TRY(cudaEventRecord(ev->spec_done, B));
+  // critical path: tail summary + scoring + top-K, then repair of the missed blocks
+  PRR_TRY(record_mark(ev->t_begin, A));
+  PRR_TRY(launch_select(p, A, hi));
+  PRR_TRY(record_mark(ev->t_select_end, A));
+  PRR_TRY(cudaEventRecord(ev->sel_done, A));
+  PRR_TRY(launch_attention(p, km, vm, 1, A, hi));
+  PRR_TRY(record_mark(ev->t_repair_end, A));
+  // spec stream: the predictor for step t+1 needs S_t only; it overlaps repair/merge
+  PRR_TRY(cudaStreamWaitEvent(B, ev->sel_done, 0));
+  PRR_TRY(record_mark(ev->t_ema_begin, B));
+  PRR_TRY(launch_ema(p, B, lo));  // the state advances even with no speculation budget
+  PRR_TRY(record_mark(ev->t_ema_end, B));
+  PRR_TRY(cudaEventRecord(ev->join, B));
+  // merge once speculation and repair are both done
+  PRR_TRY(cudaStreamWaitEvent(A, ev->spec_done, 0));
+  PRR_TRY(record_mark(ev->t_combine_begin, A));
+  PRR_TRY(launch_combine(p, A, hi));
+  PRR_TRY(record_mark(ev->t_combine_end, A));
+  PRR_TRY(cudaStreamWaitEvent(A, ev->join, 0));
 #undef PRR_TRY
   return PRR_OK;
+}
+
+prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* b, void* ws, size_t ws_bytes,
+                                 int32_t step_parity, cudaStream_t stream) {
+  if (step_parity != 0 && step_parity != 1) return PRR_ERR_INVALID_ARG;
+  Params p;
+  const prr_status st = step_params(dims, b, ws, ws_bytes, &p);
+  if (st != PRR_OK) return st;
+  if (fused_smem_bytes(p) > 227 * 1024) return PRR_ERR_SHAPE;
+  p.parity = step_parity;
+  CUtensorMap km, vm;
+  if (!make_kv_map(&km, b->k_cache, dims) || !make_kv_map(&vm, b->v_cache, dims)) return PRR_ERR_CUDA;
+  const DeviceInfo di = device_info();
+  return cuda_status(launch_fused(p, km, vm, stream, di.prio_high, di.sms, nullptr));
 }
 
 }  // extern "C"

@@ -1,0 +1,248 @@
+// prr_attn.cuh -- online-softmax statistics of ONE KV block for all G query heads of a
+// GQA group: the unit of speculation and of repair.
+//
+// PRR abstract / method summary: attention over the predicted blocks runs while the
+// selection is in flight; once the true set is known the missed blocks are attended
+// and everything is merged through online-softmax statistics.  Per block and head:
+//   m = max_i s_i,  l = sum_i 2^(s_i - m),  O = sum_i 2^(s_i - m) v_i
+// with s_i = scale*log2(e) * q.k_i (base-2 logits) over the block's tokens below n.
+// One partial per block means a predicted block that selection drops is simply never
+// merged (reuse = keep the partials of Pred n S).
+//
+// Data path (sm_100a): the block's K and V tiles ([bs][d] bf16, contiguous in the
+// cache) arrive by 3-D TMA with the 128-byte swizzle, one mbarrier each, so the
+// ldmatrix reads below are bank-conflict free.  Each staged tile is shared by all G
+// heads.  Both products run on the tensor cores with mma.m16n8k16 in swap-AB form:
+//   S^T[tok][h] = K[tok][:] . Q^T[:][h]     (M = 16 tokens, N = 8 heads, K = d)
+//   O^T[c][h]   = V^T[c][tok] . P^T[tok][h] (M = 16 channels, N = 8 heads, K = tokens)
+// The S^T accumulator fragment becomes the P^T operand fragment through movmatrix
+// (an in-register 8x8 transpose).  P is split as bf16 hi + bf16 lo (two MMAs) so the
+// PV product keeps ~16 mantissa bits.  Four warps own disjoint token slices; their O^T
+// partial sums are added in shared memory.
+#pragma once
+
+#include "prr_kernels.cuh"
+
+namespace prr {
+
+template <int D, int BS>
+struct AttnTile {
+  static constexpr int TILEB = BS * D * 2;  // one K or V tile
+  static constexpr int REGB = BS * 128;     // one 64-channel swizzle region of a tile
+  static constexpr size_t bytes = 2 * static_cast<size_t>(TILEB) + 80 * 4;  // tiles + reductions
+};
+
+// Where one block's partial goes: m/l of head h at m[h*rstride], O at O[h*ostride].
+struct PartialDst {
+  float* m;
+  float* l;
+  float* O;
+  size_t rstride;
+  size_t ostride;
+};
+
+__device__ __forceinline__ void write_empty_partial(const PartialDst& dst, int G, int D) {
+  for (int e = threadIdx.x; e < G * D; e += blockDim.x) dst.O[(e / D) * dst.ostride + (e % D)] = 0.f;
+  if (static_cast<int>(threadIdx.x) < G) {
+    dst.m[threadIdx.x * dst.rstride] = -INFINITY;
+    dst.l[threadIdx.x * dst.rstride] = 0.f;
+  }
+}
+
+// Partial of block `blk` of unit u (tokens below n).  Every thread of a 128-thread CTA
+// calls it.  `smem` is 1024-byte aligned with AttnTile::bytes free; bars[0], bars[1]
+// are initialised mbarriers (count 1) whose current phase parity is `phase` (both are
+// used once).  Returns false if a copy did not land in time (status word set).
+template <int D, int BS>
+__device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CUtensorMap* vmap, int u,
+                              int blk, int n, const PartialDst& dst, unsigned char* smem, uint64_t* bars,
+                              uint32_t phase) {
+  using L = AttnTile<D, BS>;
+  constexpr int TILEB = L::TILEB, REGB = L::REGB, NREG = D / 64;
+  constexpr int MTW = BS / 64;  // 16-token m-tiles per warp (4 warps)
+  constexpr int KS = D / 16;    // k-steps of QK^T == 16-channel tiles of PV
+  unsigned char* sK = smem;
+  unsigned char* sV = smem + TILEB;
+  float* red = reinterpret_cast<float*>(smem + 2 * TILEB);  // [0,32) max, [32,64) sum, [64,72) m, [72,80) l
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = p.G;
+
+  if (tid == 0) {
+    fence_proxy_async();  // earlier generic writes to these tiles precede the copies
+    mbar_expect_tx(&bars[0], TILEB);
+#pragma unroll
+    for (int r = 0; r < NREG; ++r) tma_load_3d(sK + r * REGB, kmap, &bars[0], r * 64, blk * BS, u);
+    mbar_expect_tx(&bars[1], TILEB);
+#pragma unroll
+    for (int r = 0; r < NREG; ++r) tma_load_3d(sV + r * REGB, vmap, &bars[1], r * 64, blk * BS, u);
+  }
+
+  // Q^T fragments (B operand of the score product): lane (g, t) holds head g,
+  // channels 16ks + 2t, +1 and 16ks + 2t + 8, +9.  Heads >= G are zero.
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t qf[KS][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(u) * G + (g < G ? g : 0)) * D);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      qf[ks][0] = g < G ? __ldg(qrow + ks * 8 + t) : 0u;
+      qf[ks][1] = g < G ? __ldg(qrow + ks * 8 + 4 + t) : 0u;
+    }
+  }
+
+  const int nv = min(BS, n - blk * BS);  // valid tokens of this block
+  if (!__syncthreads_and(mbar_wait(&bars[0], phase, p.status))) {
+    if (tid == 0) mbar_wait(&bars[1], phase, p.status);  // let the V copy land (bounded)
+    return false;
+  }
+
+  // ---- S^T = K Q^T on the tensor cores
+  const uint32_t sK_addr = smem_addr(sK), sV_addr = smem_addr(sV);
+  float sc[MTW][4];
+#pragma unroll
+  for (int mi = 0; mi < MTW; ++mi) {
+    const int mt = warp * MTW + mi;
+    sc[mi][0] = sc[mi][1] = sc[mi][2] = sc[mi][3] = 0.f;
+    const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int ch = 2 * ks + (lane >> 4);
+      const uint32_t addr = sK_addr + (ch >> 3) * REGB + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+      uint32_t a[4];
+      ldsm_x4(addr, a);
+      mma_16816(sc[mi], a, qf[ks][0], qf[ks][1]);
+    }
+  }
+  // base-2 logits; tokens >= nv masked.  sc[mi][0..1]: token 16mt+g, heads 2t, 2t+1;
+  // sc[mi][2..3]: token 16mt+g+8.
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int mi = 0; mi < MTW; ++mi) {
+    const int tok = (warp * MTW + mi) * 16 + g;
+    const bool v0 = tok < nv, v1 = tok + 8 < nv;
+    sc[mi][0] = v0 ? sc[mi][0] * p.scale_log2 : -INFINITY;
+    sc[mi][1] = v0 ? sc[mi][1] * p.scale_log2 : -INFINITY;
+    sc[mi][2] = v1 ? sc[mi][2] * p.scale_log2 : -INFINITY;
+    sc[mi][3] = v1 ? sc[mi][3] * p.scale_log2 : -INFINITY;
+    mx0 = fmaxf(mx0, fmaxf(sc[mi][0], sc[mi][2]));
+    mx1 = fmaxf(mx1, fmaxf(sc[mi][1], sc[mi][3]));
+  }
+#pragma unroll
+  for (int o = 4; o <= 16; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, o));
+  }
+  if (g == 0) {
+    red[warp * 8 + 2 * t] = mx0;
+    red[warp * 8 + 2 * t + 1] = mx1;
+  }
+  __syncthreads();
+  float m0 = red[2 * t], m1 = red[2 * t + 1];
+#pragma unroll
+  for (int w = 1; w < 4; ++w) {
+    m0 = fmaxf(m0, red[w * 8 + 2 * t]);
+    m1 = fmaxf(m1, red[w * 8 + 2 * t + 1]);
+  }
+
+  // ---- P = 2^(s - m), split hi/lo, transposed into B fragments
+  float ls0 = 0.f, ls1 = 0.f;
+  uint32_t bh[MTW][2], bl[MTW][2];
+#pragma unroll
+  for (int mi = 0; mi < MTW; ++mi) {
+    const float p0 = exp2f(sc[mi][0] - m0), p1 = exp2f(sc[mi][1] - m1);
+    const float p2 = exp2f(sc[mi][2] - m0), p3 = exp2f(sc[mi][3] - m1);
+    ls0 += p0 + p2;
+    ls1 += p1 + p3;
+    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+    const uint32_t l01 = pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01));
+    const uint32_t l23 = pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23));
+    bh[mi][0] = movmatrix_trans(h01);
+    bh[mi][1] = movmatrix_trans(h23);
+    bl[mi][0] = movmatrix_trans(l01);
+    bl[mi][1] = movmatrix_trans(l23);
+  }
+#pragma unroll
+  for (int o = 4; o <= 16; o <<= 1) {
+    ls0 += __shfl_xor_sync(0xFFFFFFFFu, ls0, o);
+    ls1 += __shfl_xor_sync(0xFFFFFFFFu, ls1, o);
+  }
+  if (g == 0) {
+    red[32 + warp * 8 + 2 * t] = ls0;
+    red[32 + warp * 8 + 2 * t + 1] = ls1;
+  }
+
+  if (!__syncthreads_and(mbar_wait(&bars[1], phase, p.status))) return false;
+  if (nv < BS) {  // tokens past the end of the sequence: zero V so 0 * V stays 0
+    uint4* v4 = reinterpret_cast<uint4*>(sV);
+    const int rows = BS - nv;
+    for (int i = tid; i < rows * NREG * 8; i += blockDim.x) {
+      const int r = nv + i / (NREG * 8), rem = i % (NREG * 8);
+      v4[((rem >> 3) * REGB + r * 128) / 16 + (rem & 7)] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  __syncthreads();
+  if (warp == 0 && g == 0) {
+    float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      l0 += red[32 + w * 8 + 2 * t];
+      l1 += red[32 + w * 8 + 2 * t + 1];
+    }
+    red[64 + 2 * t] = m0;
+    red[64 + 2 * t + 1] = m1;
+    red[72 + 2 * t] = l0;
+    red[72 + 2 * t + 1] = l1;
+  }
+
+  // ---- O^T = V^T P^T on the tensor cores
+  float oacc[KS][4];
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) oacc[dt][0] = oacc[dt][1] = oacc[dt][2] = oacc[dt][3] = 0.f;
+#pragma unroll
+  for (int mi = 0; mi < MTW; ++mi) {
+    const int mt = warp * MTW + mi;
+    const int row = mt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      const int ch = 2 * dt + ((lane >> 3) & 1);
+      const uint32_t addr = sV_addr + (ch >> 3) * REGB + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+      uint32_t a[4];
+      ldsm_x4_trans(addr, a);
+      mma_16816(oacc[dt], a, bh[mi][0], bh[mi][1]);
+      mma_16816(oacc[dt], a, bl[mi][0], bl[mi][1]);
+    }
+  }
+  // per-warp O^T into the (dead) K tile: redO[warp][h][c ^ 4h], conflict-free
+  float* redO = reinterpret_cast<float*>(sK);
+#pragma unroll
+  for (int dt = 0; dt < KS; ++dt) {
+    const int c0 = dt * 16 + g;
+    redO[(warp * 8 + 2 * t) * D + (c0 ^ (8 * t))] = oacc[dt][0];
+    redO[(warp * 8 + 2 * t + 1) * D + (c0 ^ (8 * t + 4))] = oacc[dt][1];
+    redO[(warp * 8 + 2 * t) * D + ((c0 + 8) ^ (8 * t))] = oacc[dt][2];
+    redO[(warp * 8 + 2 * t + 1) * D + ((c0 + 8) ^ (8 * t + 4))] = oacc[dt][3];
+  }
+  __syncthreads();
+  constexpr int C4 = D / 4;
+  for (int e = tid; e < G * C4; e += blockDim.x) {
+    const int h = e / C4, c4 = e % C4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float4 v = *reinterpret_cast<const float4*>(redO + (w * 8 + h) * D + ((4 * c4) ^ (4 * h)));
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    reinterpret_cast<float4*>(dst.O + h * dst.ostride)[c4] = acc;
+  }
+  if (tid < G) {
+    dst.m[tid * dst.rstride] = red[64 + tid];
+    dst.l[tid * dst.rstride] = red[72 + tid];
+  }
+  fence_proxy_async();  // this thread's generic writes to the tiles precede later copies
+  return true;
+}
+
+}  // namespace prr

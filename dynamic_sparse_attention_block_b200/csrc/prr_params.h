@@ -20,24 +20,16 @@ enum : int {
 // A bounded wait gives up after this long (one second).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
-// Merge tickets: the contributions of one (sequence, KV head) add up to this value
-// exactly once, and whoever brings the counter there runs the LSE merge.
-constexpr unsigned kMergeTarget = 1u << 30;
-
-enum : int { MODE_STANDALONE = 0, MODE_STEP = 1 };
-
 // Byte offsets inside the caller-owned workspace (all 256-byte aligned).
 struct WsLayout {
   size_t status;     // int32 status word
   size_t sel_cnt;    // uint32 [units] chunk tickets of the selection kernel
-  size_t merge_cnt;  // uint32 [units] merge tickets
-  size_t cand;       // uint64 [units][max_chunks][list_len] per-chunk top lists
+  size_t keys;       // uint32 [units][maxnb] order-preserving block-score keys
   size_t rm;         // float [units*G][K] repair partial max (base-2 logits)
   size_t rl;         // float [units*G][K] repair partial sum
   size_t rO;         // float [units*G][K][d] repair partial numerator
+  size_t ctl;        // uint32 [2][16 + 4*units] control words of the fused step
   size_t total;
-  int max_chunks;
-  int list_len;
 };
 
 struct Params {
@@ -45,11 +37,15 @@ struct Params {
   int B, Hq, Hkv, G, d, bs, cap, K, P, maxnb, units;
   float scale_log2;  // softmax scale * log2(e): logits are handled in base 2
   double alpha;      // EMA decay
-  int mode;
+  int append_summary;  // selection also folds token seq_lens[b]-1 into its block summary
   // selection geometry
   int chunk_blocks;  // blocks per selection CTA (multiple of 32)
   int nchunks;       // selection CTAs per unit
-  int list_len;      // 32 * keys per lane
+  // fused single-launch step
+  int parity;        // which copy of the control words this launch uses
+  int ctl_words;     // words per copy
+  int fchunks;       // SEL items per unit
+  int fused_region;  // bytes of the per-CTA shared-memory union
   // caller buffers (any may be null when the kernel does not use it)
   const uint16_t* q;        // [B][Hq][d] bf16
   const uint16_t* kc;       // [B][Hkv][cap][d] bf16
@@ -71,11 +67,12 @@ struct Params {
   // workspace views
   int* status;
   unsigned* sel_cnt;
-  unsigned* merge_cnt;
-  uint64_t* cand;
+  uint32_t* keys;
   float* rm;
   float* rl;
   float* rO;
+  unsigned* ctl;
+  unsigned long long* trace;  // optional: per fused item {start ns, end ns, sm, item}
   // summary update range (null: append of token seq_lens[b]-1)
   const int* tok_begin;
   const int* tok_end;

@@ -1,0 +1,158 @@
+// prr_select.cuh -- CTA-wide ranking primitives: radix selection of the k-th largest
+// 32-bit key, and bitmap-based selection and ordered emission.
+//
+// Ranking order everywhere: larger key first, ties broken by the lower index.  The
+// top-k set is therefore {key > T} plus the lowest-index entries with key == T, where
+// T is the k-th largest key (with multiplicity).  T is found MSB-first, 8 bits per
+// pass, from a shared-memory histogram.  Sets are then held as bitmaps (one ballot per
+// 32 entries); trimming the ties and writing a set in ascending index order take one
+// warp, popcounts and a shuffle prefix sum.  These routines run once per step on the
+// critical path, so they use few barriers and no CTA-wide scans.  Every thread of the
+// CTA must call the functions that contain __syncthreads (marked "CTA").
+#pragma once
+
+#include <cstdint>
+
+namespace prr {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// Inclusive warp prefix sum.
+__device__ __forceinline__ int warp_inclusive_sum(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+// CTA.  k-th largest key (1 <= k <= number of members) among entries i < n with
+// member(i).  Returns T; *n_gt = number of members with key > T.  `hist`: 256 unsigned
+// of shared scratch; `bc`: 2 ints of shared scratch.
+template <typename KeyFn, typename MemberFn>
+__device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, unsigned* hist, int* bc,
+                                      int* n_gt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NT = blockDim.x;
+  uint32_t prefix = 0u, pmask = 0u;
+  int krem = k, above_total = 0;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += NT) hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += NT) {
+      if (member(i)) {
+        const uint32_t kv = key(i);
+        if ((kv & pmask) == prefix) atomicAdd(&hist[(kv >> shift) & 0xFFu], 1u);
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns bins 255-8l down to 248-8l, so lanes run from the top bin down
+      unsigned c[8];
+      int s = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[255 - 8 * lane - j];
+        s += static_cast<int>(c[j]);
+      }
+      const int inc = warp_inclusive_sum(s);
+      const int exc = inc - s;
+      if (exc < krem && inc >= krem) {
+        int acc = exc;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (acc + static_cast<int>(c[j]) >= krem) {
+            bc[0] = 255 - 8 * lane - j;
+            bc[1] = acc;
+            break;
+          }
+          acc += static_cast<int>(c[j]);
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t dsel = static_cast<uint32_t>(bc[0]);
+    const int above = bc[1];
+    above_total += above;
+    krem -= above;
+    prefix |= dsel << shift;
+    pmask |= 0xFFu << shift;
+  }
+  __syncthreads();  // bc / hist reusable
+  *n_gt = above_total;
+  return prefix;
+}
+
+// CTA.  Bitmap `bm` (ceil(n/32) words) of the entries with cmp(i) > 0 plus the
+// `take_equal` lowest-index entries with cmp(i) == 0 (cmp(i) < 0: not selected).
+// `eq` is scratch of the same size.  On return bm is complete and visible to all.
+template <typename CmpFn>
+__device__ void select_bitmap(int n, int take_equal, CmpFn cmp, unsigned* bm, unsigned* eq) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int W = (n + 31) / 32;
+  for (int wd = warp; wd < W; wd += nw) {
+    const int i = wd * 32 + lane;
+    const int c = i < n ? cmp(i) : -1;
+    const unsigned gt = __ballot_sync(kFull, c > 0);
+    const unsigned e = __ballot_sync(kFull, c == 0);
+    if (lane == 0) {
+      bm[wd] = gt;
+      eq[wd] = e;
+    }
+  }
+  __syncthreads();
+  if (warp == 0 && take_equal > 0) {  // the first take_equal tie bits, in index order
+    int base = 0;
+    for (int w0 = 0; w0 < W; w0 += 32) {
+      const int wd = w0 + lane;
+      unsigned e = wd < W ? eq[wd] : 0u;
+      const int c = __popc(e);
+      const int inc = warp_inclusive_sum(c);
+      const int exc = base + inc - c;
+      if (e && exc < take_equal) {
+        const int need = take_equal - exc;
+        unsigned keepm = e;
+        if (need < c) {
+          keepm = 0u;
+          for (int r = 0; r < need; ++r) {
+            const unsigned low = e & (0u - e);
+            keepm |= low;
+            e ^= low;
+          }
+        }
+        bm[wd] |= keepm;
+      }
+      base += __shfl_sync(kFull, inc, 31);
+      if (base >= take_equal) break;
+    }
+  }
+  __syncthreads();
+}
+
+// One warp.  Write the set bits of bm[0..W) (optionally masked by ~exclude) as
+// ascending indices to out[0..), then -1 up to `cap`.  Returns the count.
+__device__ __forceinline__ int warp_emit_bitmap(const unsigned* bm, const unsigned* exclude, int W, int* out,
+                                                int cap) {
+  const int lane = threadIdx.x & 31;
+  int base = 0;
+  for (int w0 = 0; w0 < W; w0 += 32) {
+    const int wd = w0 + lane;
+    unsigned b = wd < W ? (exclude ? (bm[wd] & ~exclude[wd]) : bm[wd]) : 0u;
+    const int c = __popc(b);
+    const int inc = warp_inclusive_sum(c);
+    int pos = base + inc - c;
+    while (b) {
+      const int bit = __ffs(b) - 1;
+      if (pos < cap) out[pos] = wd * 32 + bit;
+      ++pos;
+      b &= b - 1u;
+    }
+    base += __shfl_sync(kFull, inc, 31);
+  }
+  for (int e = base + lane; e < cap; e += 32) out[e] = -1;
+  return base;
+}
+
+}  // namespace prr

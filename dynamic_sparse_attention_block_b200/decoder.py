@@ -56,11 +56,13 @@ class PRRDecoder:
         lo, hi = torch.cuda.Stream.priority_range()
         self.select_stream = torch.cuda.Stream(device=dev, priority=hi)
         self.spec_stream = torch.cuda.Stream(device=dev, priority=lo)
-        self.ev_fork = torch.cuda.Event()
-        self.ev_join = torch.cuda.Event()
-        self.ev_fork.record(self.select_stream)  # materialise the handles
-        self.ev_join.record(self.select_stream)
+        # stream-ordering events of the step (torch creates a handle on first record)
+        self.step_events = {name: torch.cuda.Event() for name in _abi.STEP_EVENTS}
+        for ev in self.step_events.values():
+            ev.record(self.select_stream)
         self.parity = 0  # which pred buffer holds Pred_t
+        self.fused_parity = 0  # control-word copy of the next fused launch
+        self.trace = None      # optional per-item timeline of fused launches (enable_trace)
 
     # ------------------------------------------------------------------ views
     @property
@@ -81,14 +83,31 @@ class PRRDecoder:
         b.keep = self.keep.data_ptr()
         b.part_m, b.part_l, b.part_O = self.part_m.data_ptr(), self.part_l.data_ptr(), self.part_O.data_ptr()
         b.out, b.lse = self.out.data_ptr(), self.lse.data_ptr()
+        b.trace = self.trace.data_ptr() if self.trace is not None else None
         return b
 
     def events(self, timing: Optional[dict] = None) -> _abi.PrrStepEvents:
+        """Step events; `timing` maps names of _abi.TIMING_MARKS to timing-enabled
+        torch events that have been recorded once (so that their handles exist)."""
         e = _abi.PrrStepEvents()
-        e.fork, e.join = self.ev_fork.cuda_event, self.ev_join.cuda_event
+        for name, ev in self.step_events.items():
+            setattr(e, name, ev.cuda_event)
         for name, ev in (timing or {}).items():
+            if name not in _abi.TIMING_MARKS:
+                raise ValueError(f"unknown timing mark {name}")
             setattr(e, name, ev.cuda_event)
         return e
+
+    def fused_items(self) -> dict:
+        """Work-item counts of one fused launch, in queue order."""
+        d = self.dims
+        return {"sel": d.units * -(-d.maxnb // 128), "spec": d.units * d.P, "repair": d.units * d.K,
+                "ema": d.units, "combine": d.units * d.G}
+
+    def enable_trace(self, on: bool = True) -> None:
+        """Record start/end times of every work item of the fused launches."""
+        self.trace = torch.zeros((sum(self.fused_items().values()), 4), dtype=torch.int64,
+                                 device=self.device) if on else None
 
     # ------------------------------------------------------------------ setup
     def prefill(self, k: torch.Tensor, v: torch.Tensor, n0: int) -> None:
@@ -127,6 +146,20 @@ class PRRDecoder:
                 self.q.copy_(q)
         _abi.prr_decode_step(self.dims, self.buffers(), self.ws, self.select_stream,
                              self.spec_stream, self.events(timing))
+        if swap and self.dims.P > 0:
+            self.parity ^= 1
+
+    def step_fused(self, q: Optional[torch.Tensor] = None, stream=None, swap: bool = True,
+                   parity: Optional[int] = None) -> None:
+        """The same step as one persistent launch on `stream` (default: select_stream)."""
+        st = stream or self.select_stream
+        if q is not None:
+            with torch.cuda.stream(st):
+                self.q.copy_(q)
+        par = self.fused_parity if parity is None else parity
+        _abi.prr_decode_step_fused(self.dims, self.buffers(), self.ws, par, st)
+        if parity is None:
+            self.fused_parity ^= 1
         if swap and self.dims.P > 0:
             self.parity ^= 1
 

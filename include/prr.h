@@ -105,19 +105,31 @@ typedef struct {
   float* part_O;
   float* out;
   float* lse;
+  /* Optional (NULL: off).  prr_decode_step_fused records, for every work item i of the
+   * launch, trace[4i..4i+3] = {start ns, end ns, (SM id << 32) | CTA, i} (%globaltimer).
+   * Items, in order: units*ceil(maxnb/128) selection chunks, units*P speculative
+   * slots, units*K repair slots, units predictor updates, units*G merges. */
+  unsigned long long* trace;
 } prr_step_buffers;
 
-/* Events of one decode step.  fork and join are required (any flags); the timing
- * marks are optional (NULL to skip) and, when given, must be created with timing. */
+/* Events of one decode step.  fork, sel_done, spec_done and join are required (any
+ * flags); they order the two streams.  The timing marks are optional (NULL to skip);
+ * when given they must be created with timing enabled, and under stream capture they
+ * become event-record nodes of the graph. */
 typedef struct {
-  cudaEvent_t fork;             /* recorded on select_stream, waited by spec_stream */
-  cudaEvent_t join;             /* recorded on spec_stream, waited by select_stream */
-  cudaEvent_t t_begin;          /* select_stream: before the summary update */
-  cudaEvent_t t_select_end;     /* select_stream: after selection */
-  cudaEvent_t t_repair_end;     /* select_stream: after repair */
-  cudaEvent_t t_ema_end;        /* select_stream: after the EMA predictor */
-  cudaEvent_t t_spec_begin;     /* spec_stream: before speculation */
-  cudaEvent_t t_spec_end;       /* spec_stream: after speculation */
+  cudaEvent_t fork;          /* select_stream -> spec_stream: start of the step */
+  cudaEvent_t sel_done;      /* select_stream -> spec_stream: S_t is known (predictor may run) */
+  cudaEvent_t spec_done;     /* spec_stream -> select_stream: speculative partials written */
+  cudaEvent_t join;          /* spec_stream -> select_stream: end of the spec stream's work */
+  cudaEvent_t t_begin;       /* select_stream: before selection */
+  cudaEvent_t t_select_end;  /* select_stream: after selection */
+  cudaEvent_t t_repair_end;  /* select_stream: after repair */
+  cudaEvent_t t_combine_begin; /* select_stream: before the LSE merge (after its wait) */
+  cudaEvent_t t_combine_end; /* select_stream: after the LSE merge */
+  cudaEvent_t t_spec_begin;  /* spec_stream: before speculation */
+  cudaEvent_t t_spec_end;    /* spec_stream: after speculation */
+  cudaEvent_t t_ema_begin;   /* spec_stream: before the predictor */
+  cudaEvent_t t_ema_end;     /* spec_stream: after the predictor */
 } prr_step_events;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -127,8 +139,8 @@ int prr_version(void);
 const char* prr_status_string(prr_status s);
 
 /* Bytes of workspace the calls below need for these dims (0 if the dims are
- * unsupported).  The workspace holds the status word, selection and merge tickets,
- * per-chunk candidate lists and the repair partials. */
+ * unsupported).  The workspace holds the status word, the selection tickets, one
+ * 32-bit score key per block and the repair partials. */
 size_t prr_workspace_bytes(const prr_dims* dims);
 
 /* Zero-fill a workspace (required once before first use, and after a device error).
@@ -203,19 +215,32 @@ prr_status prr_repair_merge(const prr_dims* dims, const uint16_t* q, const uint1
                             cudaStream_t stream);
 
 /* One full decode step (a1-a7) after the caller appended the step's token:
- *   select_stream: summary update -> selection -> repair -> EMA predictor
- *   spec_stream:   speculation over buf->pred (runs concurrently with selection)
- * Whichever of selection, speculation and repair finishes a (sequence, KV head) last
- * runs its LSE merge, so no kernel waits for another.  On return the work is enqueued;
- * select_stream waits for spec_stream at the end (event join), so completion of
- * select_stream means the step is done.  Selection, repair and the summary update run
- * at the highest stream priority; speculation and the predictor at the lowest.  The
- * caller swaps pred/pred_next between steps.  Capturable in a CUDA graph (no
- * allocation, no synchronisation).  PRR method summary: speculation overlaps
- * selection; the speculative budget keeps it off the critical path. */
+ *   select_stream: [tail summary + scoring + top-K] -> repair -> (wait spec) LSE merge
+ *   spec_stream:   speculation over buf->pred -> (wait selection) EMA predictor
+ * Speculation runs while selection is in flight; the predictor for step t+1 runs while
+ * the missed blocks are repaired and merged.  Selection, repair and merge are launched
+ * at the highest stream priority, speculation and prediction at the lowest.  On return
+ * the work is enqueued; select_stream waits for spec_stream at the end (event join), so
+ * completion of select_stream means the step is done.  The caller swaps pred/pred_next
+ * between steps.  No allocation and no synchronisation, so the step can be captured
+ * into a CUDA graph (after one uncaptured call on the device).  PRR method summary:
+ * speculation overlaps selection and is kept off the critical path. */
 prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* buf, void* ws,
                            size_t ws_bytes, cudaStream_t select_stream, cudaStream_t spec_stream,
                            const prr_step_events* events);
+
+/* The same decode step (a1-a7) in ONE persistent launch on `stream`.  Resident CTAs
+ * take work from a queue ordered selection -> speculation -> repair -> predictor ->
+ * merge; speculation overlaps selection inside the launch, a speculative block that
+ * selection has already dropped is skipped, and dependent work waits (bounded) only on
+ * earlier queue entries.  step_parity (0 or 1) must alternate between consecutive
+ * calls that share `ws`: each launch uses one copy of the workspace control words and
+ * clears the other for the next launch.  Same buffers, results and error behaviour as
+ * prr_decode_step; capturable in a CUDA graph (one graph per parity).
+ * PRR abstract / method summary: speculation overlaps selection and stays off the
+ * critical path; repair merges the missed blocks without recomputation. */
+prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* buf, void* ws,
+                                 size_t ws_bytes, int32_t step_parity, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -45,11 +45,13 @@ def appended_tokens(w: W.Workload, steps: int):
 
 
 def run_parity(w: W.Workload, steps: int, units: Optional[Sequence[Tuple[int, int]]] = None,
-               forced: Optional[Tuple[float, int]] = None, graph: bool = False) -> Report:
+               forced: Optional[Tuple[float, int]] = None, graph: bool = False,
+               mode: str = "fused") -> Report:
     """Compare `steps` decode steps.  `units` samples the (b, kvh) pairs the oracle
     follows (default: all).  `forced` = (overlap, level) replaces the predictor's output
     with a predicted set forced to that overlap with the oracle's true set (all units
-    are then followed)."""
+    are then followed).  `mode` selects the step implementation: "fused" (one
+    persistent launch) or "streams" (two streams, one launch per kernel)."""
     o = OR.default()
     all_units = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     if units is None or forced is not None:
@@ -76,20 +78,24 @@ def run_parity(w: W.Workload, steps: int, units: Optional[Sequence[Tuple[int, in
             dec.pred.copy_(torch.from_numpy(pred_host))
         pred_used = dec.pred.clone()
         if graph and t >= 2:  # steps 0-1 run eagerly first (warm-up before capture)
-            par = dec.parity
-            if par not in graphs:
-                # capture after eager warm-up steps have run
+            key = (dec.parity, dec.fused_parity)
+            if key not in graphs:
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=dec.select_stream):
-                    dec.step(swap=False)
-                graphs[par] = g
-                dec.q.copy_(q_dev)
-                torch.cuda.synchronize()
+                    if mode == "fused":
+                        dec.step_fused(swap=False, parity=dec.fused_parity)
+                    else:
+                        dec.step(swap=False)
+                graphs[key] = g
             dec.q.copy_(q_dev)
             torch.cuda.synchronize()
-            graphs[par].replay()
+            graphs[key].replay()
+            if mode == "fused":
+                dec.fused_parity ^= 1
             if dims.P > 0:
                 dec.parity ^= 1
+        elif mode == "fused":
+            dec.step_fused(q_dev)
         else:
             dec.step(q_dev)
         torch.cuda.synchronize()

@@ -259,35 +259,51 @@ def _assert_ok(rep):
     assert rep.max_out_err <= OUT_TOL and rep.max_lse_rel <= LSE_RTOL
 
 
-def test_decode_tiny_all_steps():
+MODES = ("fused", "streams")
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_decode_tiny_all_steps(mode):
     """Tiny workload (1 KV head x 4 query heads, d 64, 4096 tokens, 16 steps), every step."""
-    _assert_ok(run_parity(W.workload("tiny"), steps=16))
+    _assert_ok(run_parity(W.workload("tiny"), steps=16, mode=mode))
 
 
-def test_decode_tiny_graph_replay():
-    """Same trajectory with the step captured once per Pred parity in a CUDA graph."""
-    _assert_ok(run_parity(W.workload("tiny"), steps=8, graph=True))
+@pytest.mark.parametrize("mode", MODES)
+def test_decode_tiny_graph_replay(mode):
+    """Same trajectory with the step captured once per parity in a CUDA graph."""
+    _assert_ok(run_parity(W.workload("tiny"), steps=8, graph=True, mode=mode))
 
 
-def test_decode_llama8b_32k():
+@pytest.mark.parametrize("mode", MODES)
+def test_decode_llama8b_32k(mode):
     """Llama-3.1-8B-shaped layer at 32K (bench workload), all 8 KV heads, 12 steps, graphs."""
-    _assert_ok(run_parity(W.workload("llama8b_32k"), steps=12, graph=True))
+    _assert_ok(run_parity(W.workload("llama8b_32k"), steps=12, graph=True, mode=mode))
 
 
-def test_decode_ragged_small():
+@pytest.mark.parametrize("mode", MODES)
+def test_decode_ragged_small(mode):
     """Small ragged shapes: context not a multiple of the block, K > some nb, G = 2."""
     w = W.workload("tiny").with_(name="ragged", B=3, Hq=6, Hkv=3, d=128, N0=1000, bs=64, K=20,
                                  P=12, steps=40, walk_p=0.7)
-    _assert_ok(run_parity(w, steps=40))
+    _assert_ok(run_parity(w, steps=40, mode=mode))
     w2 = w.with_(N0=130, bs=128, K=8, P=8, steps=5)  # K > nb for the first steps
-    _assert_ok(run_parity(w2, steps=5))
+    _assert_ok(run_parity(w2, steps=5, mode=mode))
 
 
-def test_decode_repair_sweep_small():
+@pytest.mark.parametrize("mode", MODES)
+def test_decode_no_speculation(mode):
+    """Budget P = 0: every selected block is repaired; the predictor is idle."""
+    w = W.workload("tiny").with_(name="no_spec", B=2, Hq=8, Hkv=2, d=128, N0=3000, bs=64, K=16,
+                                 P=0, steps=6)
+    _assert_ok(run_parity(w, steps=6, mode=mode))
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_decode_repair_sweep_small(mode):
     """Gaussian q/k/v with forced predictor overlap at every level (reduced context)."""
     w = W.workload("repair_sweep_64k").with_(B=2, N0=8192)
     for level, ov in enumerate(w.forced_overlaps):
-        _assert_ok(run_parity(w, steps=3, forced=(ov, level)))
+        _assert_ok(run_parity(w, steps=3, forced=(ov, level), mode=mode))
 
 
 @pytest.mark.parametrize("name,steps,units", [
@@ -295,8 +311,9 @@ def test_decode_repair_sweep_small():
     ("long_512k", 3, [(0, 0), (2, 5), (3, 7)]),
 ])
 def test_decode_full_size_sampled(name, steps, units):
-    """Full-size workloads, the whole batch on the GPU, sampled units in the oracle."""
-    _assert_ok(run_parity(W.workload(name), steps=steps, units=units))
+    """Full-size workloads, the whole batch on the GPU (fused step, graphs), sampled
+    units in the oracle."""
+    _assert_ok(run_parity(W.workload(name), steps=steps, units=units, graph=False))
 
 
 def test_decode_repair_sweep_full_size():

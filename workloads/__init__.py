@@ -69,7 +69,8 @@ class Workload:
         return self.B * self.Hkv
 
     def seed_of(self, b: int) -> int:
-        return b if self.per_seq_seed else self.seed
+        # per-sequence seeds are b (plus an offset that distinguishes replicas)
+        return b + self.seed if self.per_seq_seed else self.seed
 
     def cap_tokens(self, extra_steps: int = 0) -> int:
         return self.N0 + self.steps + extra_steps
