@@ -31,18 +31,21 @@ namespace prr {
 constexpr int kFusedChunk = 128;  // blocks per SEL item (4 warps x 32 rows)
 
 struct FusedCtl {
-  unsigned* work;      // next item
-  unsigned* abort;     // set on a timed-out wait
-  unsigned* sel_cnt;   // [units] finished SEL chunks
-  unsigned* sel_done;  // [units] S_t published
-  unsigned* target;    // [units] active speculative slots + missed blocks
-  unsigned* done_cnt;  // [units] finished speculative + repair items
+  unsigned* work;        // next item
+  unsigned* abort;       // set on a timed-out wait
+  unsigned* sel_loaded;  // SEL items whose summary tile has landed
+  unsigned* sel_finished;  // units whose S_t is published
+  unsigned* sel_cnt;     // [units] finished SEL chunks
+  unsigned* sel_done;    // [units] S_t published
+  unsigned* p_act;       // [units] active speculative slots (published with S_t)
+  unsigned* spec_done;   // [units] finished (or skipped) speculative items
+  unsigned* rep_done;    // [units] finished repair items
 };
 
 __device__ __forceinline__ FusedCtl ctl_view(const Params& p, int parity) {
   unsigned* b = p.ctl + static_cast<size_t>(parity) * p.ctl_words;
   const int U = p.units;
-  return FusedCtl{b, b + 1, b + 16, b + 16 + U, b + 16 + 2 * U, b + 16 + 3 * U};
+  return FusedCtl{b, b + 1, b + 2, b + 3, b + 16, b + 16 + U, b + 16 + 2 * U, b + 16 + 3 * U, b + 16 + 4 * U};
 }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -142,6 +145,7 @@ __device__ void sel_item(const Params& p, const FusedCtl& C, int u, int chunk, u
       return;
     }
   }
+  if (tid == 0) atomicAdd(C.sel_loaded, 1u);  // this chunk no longer needs bandwidth
   const int first = c0 + 32 * warp;
   const int rows = min(32, cnt - 32 * warp);
   if (rows > 0) {
@@ -163,9 +167,10 @@ __device__ void sel_item(const Params& p, const FusedCtl& C, int u, int chunk, u
   __threadfence();  // every thread's outputs are visible before S_t is published
   __syncthreads();
   if (tid == 0) {
-    C.target[u] = static_cast<unsigned>(f.p_active + f.n_missed);
+    C.p_act[u] = static_cast<unsigned>(f.p_active);
     __threadfence();
     atomicExch(C.sel_done + u, 1u);
+    atomicAdd(C.sel_finished, 1u);
   }
 }
 
@@ -229,6 +234,10 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
       const int nb = (n + BS - 1) / BS;
       const int blk = p.pred[static_cast<size_t>(u) * p.P + j];
       if (blk >= 0 && blk < nb) {
+        // speculation has slack; selection is on the critical path.  Gate 1: wait until
+        // every selection tile has landed; gate 2: until every unit's S_t is published.
+        if (p.spec_gate == 1) wait_geq(C.sel_loaded, static_cast<unsigned>(n_sel), C, p.status, sh);
+        if (p.spec_gate == 2) wait_geq(C.sel_finished, static_cast<unsigned>(U), C, p.status, sh);
         if (tid == 0) sh[3] = (ld_acquire(C.sel_done + u) != 0u &&
                                __ldcg(p.keep + static_cast<size_t>(u) * p.P + j) == 0) ? 1 : 0;
         __syncthreads();
@@ -241,7 +250,7 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
             atomicExch(C.abort, 1u);
           ph_attn ^= 1u;
         }
-        count_done(C.done_cnt + u);
+        count_done(C.spec_done + u);
       }
       __syncthreads();
       if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
@@ -267,7 +276,7 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
             if (tid == 0) report(p.status, kDevBadMissed);
             write_empty_partial(dst, p.G, D);
           }
-          count_done(C.done_cnt + u);
+          count_done(C.rep_done + u);
         }
       }
       __syncthreads();
@@ -285,8 +294,11 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
     {  // LSE merge of (unit, head)
       const int u = it / p.G, h = it % p.G;
       if (wait_geq(C.sel_done + u, 1u, C, p.status, sh)) {
-        const unsigned tgt = __ldcg(C.target + u);
-        if (wait_geq(C.done_cnt + u, tgt, C, p.status, sh)) combine_head<D>(p, u, h, smem);
+        const unsigned pa = __ldcg(C.p_act + u);
+        const unsigned nm = static_cast<unsigned>(min(max(__ldcg(p.n_missed + u), 0), p.K));
+        // fold the speculative partials as soon as they are all written, then the repairs
+        if (wait_geq(C.spec_done + u, pa, C, p.status, sh))
+          combine_head<D>(p, u, h, smem, [&] { return wait_geq(C.rep_done + u, nm, C, p.status, sh); });
       }
       __syncthreads();
       if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();

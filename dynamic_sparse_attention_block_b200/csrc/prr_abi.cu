@@ -55,7 +55,7 @@ WsLayout layout_for(const prr_dims* d) {
   L.rO = off;
   off = align256(off + 4 * units * G * d->K * d->d);
   L.ctl = off;
-  off = align256(off + 4 * 2 * (16 + 4 * units));
+  off = align256(off + 4 * 2 * (16 + 5 * units));
   L.total = off;
   return L;
 }
@@ -132,7 +132,15 @@ Params base_params(const prr_dims* d, void* ws) {
     p.rO = reinterpret_cast<float*>(w + L.rO);
     p.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
   }
-  p.ctl_words = 16 + 4 * p.units;
+  p.ctl_words = 16 + 5 * p.units;
+  {
+    static int gate = -1;  // PRR_SPEC_GATE in {0, 1, 2} overrides the speculation gate
+    if (gate < 0) {
+      const char* e = std::getenv("PRR_SPEC_GATE");
+      gate = (e && e[0] >= '0' && e[0] <= '2') ? e[0] - '0' : 1;
+    }
+    p.spec_gate = gate;
+  }
   return p;
 }
 

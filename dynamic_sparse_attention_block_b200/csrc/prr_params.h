@@ -28,7 +28,7 @@ struct WsLayout {
   size_t rm;         // float [units*G][K] repair partial max (base-2 logits)
   size_t rl;         // float [units*G][K] repair partial sum
   size_t rO;         // float [units*G][K][d] repair partial numerator
-  size_t ctl;        // uint32 [2][16 + 4*units] control words of the fused step
+  size_t ctl;        // uint32 [2][16 + 5*units] control words of the fused step
   size_t total;
 };
 
@@ -46,6 +46,7 @@ struct Params {
   int ctl_words;     // words per copy
   int fchunks;       // SEL items per unit
   int fused_region;  // bytes of the per-CTA shared-memory union
+  int spec_gate;     // speculative items wait: 0 no, 1 selection tiles landed, 2 all S_t published
   // caller buffers (any may be null when the kernel does not use it)
   const uint16_t* q;        // [B][Hq][d] bf16
   const uint16_t* kc;       // [B][Hkv][cap][d] bf16

@@ -23,6 +23,29 @@ __device__ unsigned long long g_phase[2][4096][8];
   } while (0)
 #endif
 
+// ------------------------------------------------------------------ batched loads
+//
+// Copy n 32-bit words (global, written by other CTAs: read through L2) into shared
+// memory with kBatch loads in flight per thread before any is consumed; a plain loop
+// would wait one memory round trip per element.
+constexpr int kBatch = 16;
+
+__device__ __forceinline__ void load_words_cg(uint32_t* dst, const uint32_t* src, int n) {
+  for (int base = 0; base < n; base += kBatch * static_cast<int>(blockDim.x)) {
+    uint32_t v[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int i = base + q * blockDim.x + threadIdx.x;
+      v[q] = i < n ? __ldcg(src + i) : 0u;
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int i = base + q * blockDim.x + threadIdx.x;
+      if (i < n) dst[i] = v[q];
+    }
+  }
+}
+
 // ------------------------------------------------------------------ block scoring
 //
 // Quest's channel-wise bound summed over the GQA group (one selection per KV head):
@@ -110,25 +133,23 @@ struct FinishOut {
 };
 
 __host__ __device__ constexpr size_t finish_scratch_bytes(int maxnb) {
-  return static_cast<size_t>(maxnb) * 4 + 4 * static_cast<size_t>((maxnb + 31) / 32) * 4 + 256 * 4 + 128 * 4 +
-         16 * 4;
+  return 256 * 4 + 128 * 4 + 16 * 4 + static_cast<size_t>(maxnb) * 4 + 3 * static_cast<size_t>((maxnb + 31) / 32) * 4;
 }
 
 __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsigned char* scratch) {
   const int tid = threadIdx.x, warp = tid >> 5;
   const int W = (p.maxnb + 31) / 32;
-  uint32_t* skeys = reinterpret_cast<uint32_t*>(scratch);
-  unsigned* bm_pred = reinterpret_cast<unsigned*>(skeys + p.maxnb);
+  unsigned* hist = reinterpret_cast<unsigned*>(scratch);  // 16-byte aligned
+  int* spred = reinterpret_cast<int*>(hist + 256);        // [128]
+  int* misc = spred + 128;                                // bc[2], counts
+  uint32_t* skeys = reinterpret_cast<uint32_t*>(misc + 16);
+  unsigned* bm_pred = skeys + p.maxnb;
   unsigned* bm_sel = bm_pred + W;
   unsigned* bm_eq = bm_sel + W;
-  unsigned* hist = bm_eq + W;
-  int* spred = reinterpret_cast<int*>(hist + 256);  // [128]
-  int* misc = spred + 128;                          // bc[2], counts
 
   PRR_PHASE(0, u, 0);
-  const uint32_t* keys_in = p.keys + static_cast<size_t>(u) * p.maxnb;
-  for (int i = tid; i < nb; i += blockDim.x) skeys[i] = __ldcg(keys_in + i);
   for (int j = tid; j < p.P; j += blockDim.x) spred[j] = p.pred[static_cast<size_t>(u) * p.P + j];
+  load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb);
   for (int i = tid; i < W; i += blockDim.x) bm_pred[i] = 0u;
   __syncthreads();
   PRR_PHASE(0, u, 1);
@@ -201,34 +222,46 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
 // ties go to the lowest block indices.
 
 __host__ __device__ constexpr size_t ema_scratch_bytes(int maxnb) {
-  return static_cast<size_t>(maxnb) * 8 + 3 * static_cast<size_t>((maxnb + 31) / 32) * 4 + 256 * 4 + 16 * 4;
+  return 256 * 4 + 16 * 4 + static_cast<size_t>(maxnb) * 8 + 3 * static_cast<size_t>((maxnb + 31) / 32) * 4;
 }
 
 __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch) {
   const int W = (p.maxnb + 31) / 32;
-  uint32_t* hi = reinterpret_cast<uint32_t*>(scratch);
+  unsigned* hist = reinterpret_cast<unsigned*>(scratch);  // 16-byte aligned
+  int* misc = reinterpret_cast<int*>(hist + 256);
+  uint32_t* hi = reinterpret_cast<uint32_t*>(misc + 16);
   uint32_t* lo = hi + p.maxnb;
   unsigned* bm = lo + p.maxnb;  // selected blocks of this step
   unsigned* bsel = bm + W;      // predicted set
   unsigned* beq = bsel + W;
-  unsigned* hist = beq + W;
-  int* misc = reinterpret_cast<int*>(hist + 256);
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   PRR_PHASE(1, u, 0);
   const int n = checked_len(p, u / p.Hkv);
   const int nb = (n + p.bs - 1) / p.bs;
   double* e = p.ema + static_cast<size_t>(u) * p.maxnb;
   const bool update = p.sel != nullptr;
 
-  // fetch the state and S_t together
-  for (int i = tid; i < nb; i += blockDim.x) {
-    const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(e[i]));
-    hi[i] = static_cast<uint32_t>(bits >> 32);
-    lo[i] = static_cast<uint32_t>(bits);
-  }
+  // fetch the state and S_t together (many loads in flight per thread)
   int sv = -1;
   if (update && tid < p.K) sv = __ldcg(p.sel + static_cast<size_t>(u) * p.K + tid);
+  for (int base = 0; base < nb; base += kBatch * static_cast<int>(blockDim.x)) {
+    double v[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int i = base + q * blockDim.x + tid;
+      v[q] = i < nb ? e[i] : 0.0;
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int i = base + q * blockDim.x + tid;
+      if (i < nb) {
+        const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(v[q]));
+        hi[i] = static_cast<uint32_t>(bits >> 32);
+        lo[i] = static_cast<uint32_t>(bits);
+      }
+    }
+  }
   for (int i = tid; i < W; i += blockDim.x) bm[i] = 0u;
   __syncthreads();
   if (update) {
@@ -266,29 +299,9 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch) 
         nb, peff, [&](int i) { return hi[i]; }, [&](int) { return true; }, hist, misc, &gt_hi);
     PRR_PHASE(1, u, 2);
     const int need = peff - gt_hi;  // taken from the entries tied on the high word
-    // do the tied entries agree on the low word?  (then the low-word pass is moot)
-    unsigned mn = 0xFFFFFFFFu, mx = 0u;
-    for (int i = tid; i < nb; i += blockDim.x)
-      if (hi[i] == Thi) {
-        mn = min(mn, lo[i]);
-        mx = max(mx, lo[i]);
-      }
-    mn = __reduce_min_sync(kFull, mn);
-    mx = __reduce_max_sync(kFull, mx);
-    if (lane == 0) {
-      misc[4 + warp] = static_cast<int>(mn);
-      misc[8 + warp] = static_cast<int>(mx);
-    }
-    __syncthreads();
-    unsigned gmin = 0xFFFFFFFFu, gmax = 0u;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
-      gmin = min(gmin, static_cast<unsigned>(misc[4 + w]));
-      gmax = max(gmax, static_cast<unsigned>(misc[8 + w]));
-    }
-    uint32_t Tlo = gmin;
-    if (gmin != gmax)
-      Tlo = radix_kth_largest(
-          nb, need, [&](int i) { return lo[i]; }, [&](int i) { return hi[i] == Thi; }, hist, misc, &gt_lo);
+    // low word among the entries tied on the high word (no pass at all when they agree)
+    const uint32_t Tlo = radix_kth_largest(
+        nb, need, [&](int i) { return lo[i]; }, [&](int i) { return hi[i] == Thi; }, hist, misc, &gt_lo);
     PRR_PHASE(1, u, 3);
     select_bitmap(
         nb, need - gt_lo,
@@ -313,123 +326,160 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch) 
 //   m* = max_j m_j,  l* = sum_j l_j 2^(m_j - m*),  out = sum_j O_j 2^(m_j - m*) / l*,
 //   lse = (m* + log2 l*) ln 2,
 // over the slots j with keep[j] = 1 (speculation) and the first n_missed repair slots.
-// 128 threads: the weighted numerator sum is split over the 4 warps, each lane one
-// float4 column with 16 slot loads in flight.
+// 128 threads.  Each warp folds its share of the slots into a running (m, l, O) state
+// (O: one float4 column per lane), rescaling when a larger max arrives, so loads never
+// wait for a CTA-wide maximum; the four warp states are combined at the end.  The
+// speculative slots are folded first; `wait_repair()` (CTA-uniform) runs between the
+// two phases, so a caller can start on the speculative part before repair is done.
 
 __host__ __device__ constexpr size_t combine_scratch_bytes(int P, int K, int D) {
-  return static_cast<size_t>(P + K) * 16 + 16 * 4 + 4 * static_cast<size_t>(D) * 4 + 32;
+  return static_cast<size_t>(P) * 12 + 16 * 4 + 4 * static_cast<size_t>(D) * 4 + 64;
 }
 
-template <int D>
-__device__ void combine_head(const Params& p, int u, int h, unsigned char* scratch) {
+struct WarpState {
+  float m;  // running max (base-2 logits), -inf when empty
+  float l;  // running sum, relative to m (meaningful in lane 0; all lanes agree)
+  float4 o; // running numerator column of this lane, relative to m
+};
+
+// Fold up to B slots (values already loaded) into the warp state.
+template <int B>
+__device__ __forceinline__ void fold_batch(WarpState& st, const float (&m)[B], const float (&l)[B],
+                                           const float4 (&o)[B]) {
+  float mb = st.m;
+#pragma unroll
+  for (int q = 0; q < B; ++q) mb = fmaxf(mb, m[q]);
+  if (mb == -INFINITY) return;
+  const float sc = st.m == -INFINITY ? 0.f : exp2f(st.m - mb);
+  st.l *= sc;
+  st.o.x *= sc;
+  st.o.y *= sc;
+  st.o.z *= sc;
+  st.o.w *= sc;
+#pragma unroll
+  for (int q = 0; q < B; ++q) {
+    const float w = m[q] == -INFINITY ? 0.f : exp2f(m[q] - mb);
+    st.l = fmaf(w, l[q], st.l);
+    st.o.x = fmaf(w, o[q].x, st.o.x);
+    st.o.y = fmaf(w, o[q].y, st.o.y);
+    st.o.z = fmaf(w, o[q].z, st.o.z);
+    st.o.w = fmaf(w, o[q].w, st.o.w);
+  }
+  st.m = mb;
+}
+
+template <int D, typename WaitFn>
+__device__ void combine_head(const Params& p, int u, int h, unsigned char* scratch, WaitFn wait_repair) {
   constexpr int C4 = D / 4;
-  const int P = p.P, K = p.K, S = P + K;
-  int* slots = reinterpret_cast<int*>(scratch);   // compacted active slots
-  float* wt = reinterpret_cast<float*>(slots + S);  // per slot: m, then weight
-  float* lv = wt + S;                               // per slot: l
-  int* actf = reinterpret_cast<int*>(lv + S);       // per slot: contributes?
-  float* red = reinterpret_cast<float*>(actf + S);  // 8 floats + count
+  constexpr int B = 8;  // slots per batch and warp: 8 float4 loads in flight per lane
+  const int P = p.P, K = p.K;
+  float* km = reinterpret_cast<float*>(scratch);  // [P] kept slot max or -inf
+  float* kl = km + P;                             // [P]
+  int* slots = reinterpret_cast<int*>(kl + P);    // [P] compacted kept slots
+  float* red = reinterpret_cast<float*>(slots + P);  // [4] m, [4] l, count
   int* count = reinterpret_cast<int*>(red + 8);
   float4* part = reinterpret_cast<float4*>((reinterpret_cast<uintptr_t>(red + 16) + 15) &
                                            ~static_cast<uintptr_t>(15));  // [4][C4]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t row = static_cast<size_t>(u) * p.G + h;
+  const bool col = lane < C4;
+  WarpState st{-INFINITY, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
 
-  // round trip 1: every slot's flag and statistics at once
-  const int nm = min(max(__ldcg(p.n_missed + u), 0), K);
-  float mloc = -INFINITY;
-  for (int s = tid; s < S; s += blockDim.x) {
-    bool act;
-    float m, l;
-    if (s < P) {
-      act = __ldcg(p.keep + static_cast<size_t>(u) * P + s) != 0;
-      m = __ldcg(p.pm + row * P + s);
-      l = __ldcg(p.pl + row * P + s);
-    } else {
-      act = (s - P) < nm;
-      m = act ? __ldcg(p.rm + row * K + (s - P)) : 0.f;
-      l = act ? __ldcg(p.rl + row * K + (s - P)) : 0.f;
-    }
-    wt[s] = act ? m : -INFINITY;
-    lv[s] = act ? l : 0.f;
-    actf[s] = act ? 1 : 0;
-    if (act) mloc = fmaxf(mloc, m);
+  // ---- speculative slots: flags and statistics in one round trip, then numerators
+  for (int j = tid; j < P; j += blockDim.x) {
+    const bool act = __ldcg(p.keep + static_cast<size_t>(u) * P + j) != 0;
+    const float m = __ldcg(p.pm + row * P + j);
+    const float l = __ldcg(p.pl + row * P + j);
+    km[j] = act ? m : -INFINITY;
+    kl[j] = act ? l : 0.f;
   }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xFFFFFFFFu, mloc, o));
-  if (lane == 0) red[warp] = mloc;
   __syncthreads();
-  const float mstar = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  float lsum = 0.f;
-  for (int s = tid; s < S; s += blockDim.x) {
-    const float w = (wt[s] == -INFINITY || mstar == -INFINITY) ? 0.f : exp2f(wt[s] - mstar);
-    wt[s] = w;
-    lsum += lv[s] * w;
-  }
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xFFFFFFFFu, lsum, o);
-  if (lane == 0) red[4 + warp] = lsum;
-  if (warp == 0) {  // compact the contributing slots
+  if (warp == 0) {
     int cnt = 0;
-    for (int base = 0; base < S; base += 32) {
-      const int s = base + lane;
-      const bool a = s < S && actf[s] != 0;
+    for (int base = 0; base < P; base += 32) {
+      const int j = base + lane;
+      const bool a = j < P && km[j] != -INFINITY;
       const unsigned mask = __ballot_sync(0xFFFFFFFFu, a);
-      if (a) slots[cnt + __popc(mask & ((1u << lane) - 1u))] = s;
+      if (a) slots[cnt + __popc(mask & ((1u << lane) - 1u))] = j;
       cnt += __popc(mask);
     }
     if (lane == 0) count[0] = cnt;
   }
   __syncthreads();
-  const float lstar = red[4] + red[5] + red[6] + red[7];
   const int ns = count[0];
-
-  // round trip 2: the numerators of the contributing slots, 16 loads in flight per lane
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  constexpr int BATCH = 16;
-  for (int s0 = warp; s0 < ns; s0 += 4 * BATCH) {
-    float4 v[BATCH];
-    float w[BATCH];
+  for (int s0 = warp; s0 < ns; s0 += 4 * B) {
+    float m[B], l[B];
+    float4 o[B];
 #pragma unroll
-    for (int q = 0; q < BATCH; ++q) {
+    for (int q = 0; q < B; ++q) {
       const int si = s0 + 4 * q;
-      v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      w[q] = 0.f;
-      if (si < ns && lane < C4) {
+      m[q] = -INFINITY;
+      l[q] = 0.f;
+      o[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (si < ns) {
         const int j = slots[si];
-        const float4* src = j < P ? reinterpret_cast<const float4*>(p.pO + (row * P + j) * D)
-                                  : reinterpret_cast<const float4*>(p.rO + (row * K + (j - P)) * D);
-        v[q] = __ldcg(src + lane);
-        w[q] = wt[j];
+        m[q] = km[j];
+        l[q] = kl[j];
+        if (col) o[q] = __ldcg(reinterpret_cast<const float4*>(p.pO + (row * P + j) * D) + lane);
       }
     }
+    fold_batch<B>(st, m, l, o);
+  }
+
+  // ---- repair slots: statistics and numerators in one round trip
+  if (wait_repair()) {
+    const int nm = min(max(__ldcg(p.n_missed + u), 0), K);
+    for (int i0 = warp; i0 < nm; i0 += 4 * B) {
+      float m[B], l[B];
+      float4 o[B];
 #pragma unroll
-    for (int q = 0; q < BATCH; ++q) {
-      acc.x = fmaf(w[q], v[q].x, acc.x);
-      acc.y = fmaf(w[q], v[q].y, acc.y);
-      acc.z = fmaf(w[q], v[q].z, acc.z);
-      acc.w = fmaf(w[q], v[q].w, acc.w);
+      for (int q = 0; q < B; ++q) {
+        const int i = i0 + 4 * q;
+        m[q] = -INFINITY;
+        l[q] = 0.f;
+        o[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < nm) {
+          m[q] = __ldcg(p.rm + row * K + i);
+          l[q] = __ldcg(p.rl + row * K + i);
+          if (col) o[q] = __ldcg(reinterpret_cast<const float4*>(p.rO + (row * K + i) * D) + lane);
+        }
+      }
+      fold_batch<B>(st, m, l, o);
     }
   }
-  if (lane < C4) part[warp * C4 + lane] = acc;
+
+  // ---- combine the four warp states
+  if (lane == 0) {
+    red[warp] = st.m;
+    red[4 + warp] = st.l;
+  }
+  if (col) part[warp * C4 + lane] = st.o;
   __syncthreads();
-  if (tid < C4) {
-    float4 o = part[tid];
+  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float L = 0.f, f[4];
 #pragma unroll
-    for (int w2 = 1; w2 < 4; ++w2) {
-      o.x += part[w2 * C4 + tid].x;
-      o.y += part[w2 * C4 + tid].y;
-      o.z += part[w2 * C4 + tid].z;
-      o.w += part[w2 * C4 + tid].w;
+  for (int w = 0; w < 4; ++w) {
+    f[w] = (red[w] == -INFINITY || M == -INFINITY) ? 0.f : exp2f(red[w] - M);
+    L = fmaf(f[w], red[4 + w], L);
+  }
+  if (tid < C4) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float4 v = part[w * C4 + tid];
+      o.x = fmaf(f[w], v.x, o.x);
+      o.y = fmaf(f[w], v.y, o.y);
+      o.z = fmaf(f[w], v.z, o.z);
+      o.w = fmaf(f[w], v.w, o.w);
     }
-    const float inv = lstar > 0.f ? 1.0f / lstar : 0.f;
+    const float inv = L > 0.f ? 1.0f / L : 0.f;
     o.x *= inv;
     o.y *= inv;
     o.z *= inv;
     o.w *= inv;
     reinterpret_cast<float4*>(p.out + row * D)[tid] = o;
   }
-  if (tid == 0) p.lse[row] = lstar > 0.f ? (mstar + log2f(lstar)) * 0.69314718055994530942f : -INFINITY;
+  if (tid == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
   __syncthreads();
 }
 

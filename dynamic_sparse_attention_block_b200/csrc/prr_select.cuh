@@ -4,7 +4,8 @@
 // Ranking order everywhere: larger key first, ties broken by the lower index.  The
 // top-k set is therefore {key > T} plus the lowest-index entries with key == T, where
 // T is the k-th largest key (with multiplicity).  T is found MSB-first, 8 bits per
-// pass, from a shared-memory histogram.  Sets are then held as bitmaps (one ballot per
+// pass, from a shared-memory histogram (plain shared atomics: cheaper here than any
+// warp-collective aggregation).  Sets are then held as bitmaps (one ballot per
 // 32 entries); trimming the ties and writing a set in ascending index order take one
 // warp, popcounts and a shuffle prefix sum.  These routines run once per step on the
 // critical path, so they use few barriers and no CTA-wide scans.  Every thread of the
@@ -29,16 +30,45 @@ __device__ __forceinline__ int warp_inclusive_sum(int v) {
 }
 
 // CTA.  k-th largest key (1 <= k <= number of members) among entries i < n with
-// member(i).  Returns T; *n_gt = number of members with key > T.  `hist`: 256 unsigned
-// of shared scratch; `bc`: 2 ints of shared scratch.
+// member(i).  Returns T; *n_gt = number of members with key > T.  `hist`: 256
+// unsigned of 16-byte aligned shared scratch; `bc`: 2 ints of shared scratch.
+// Leading bytes shared by every member key (one min/max reduction) need no pass, so
+// scores in a narrow range usually take two or three passes.
 template <typename KeyFn, typename MemberFn>
 __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, unsigned* hist, int* bc,
                                       int* n_gt) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NT = blockDim.x;
-  uint32_t prefix = 0u, pmask = 0u;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NT = blockDim.x, nw = NT >> 5;
+  unsigned kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int i = tid; i < n; i += NT) {
+    if (member(i)) {
+      const uint32_t v = key(i);
+      kmin = min(kmin, v);
+      kmax = max(kmax, v);
+    }
+  }
+  kmin = __reduce_min_sync(kFull, kmin);
+  kmax = __reduce_max_sync(kFull, kmax);
+  if (lane == 0) {
+    hist[warp] = kmin;
+    hist[32 + warp] = kmax;
+  }
+  __syncthreads();
+  unsigned gmin = 0xFFFFFFFFu, gmax = 0u;
+  for (int w = 0; w < nw; ++w) {
+    gmin = min(gmin, hist[w]);
+    gmax = max(gmax, hist[32 + w]);
+  }
+  __syncthreads();  // hist is reused below
+  if (gmin == gmax) {  // all member keys equal
+    *n_gt = 0;
+    return gmin;
+  }
+  const int skip = __clz(gmin ^ gmax) / 8;  // leading bytes common to all keys
+  uint32_t pmask = skip ? (0xFFFFFFFFu << (32 - 8 * skip)) : 0u;
+  uint32_t prefix = gmin & pmask;
   int krem = k, above_total = 0;
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (int shift = 24 - 8 * skip; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += NT) hist[i] = 0u;
     __syncthreads();
     for (int i = tid; i < n; i += NT) {
@@ -49,26 +79,31 @@ __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, 
     }
     __syncthreads();
     if (warp == 0) {
-      // lane l owns bins 255-8l down to 248-8l, so lanes run from the top bin down
-      unsigned c[8];
-      int s = 0;
+      // lane l owns bins 8l..8l+7; suffix sums run from the top bin down
+      const uint4 a = reinterpret_cast<const uint4*>(hist)[2 * lane];
+      const uint4 b = reinterpret_cast<const uint4*>(hist)[2 * lane + 1];
+      const int c[8] = {static_cast<int>(a.x), static_cast<int>(a.y), static_cast<int>(a.z), static_cast<int>(a.w),
+                        static_cast<int>(b.x), static_cast<int>(b.y), static_cast<int>(b.z), static_cast<int>(b.w)};
+      int sum = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        c[j] = hist[255 - 8 * lane - j];
-        s += static_cast<int>(c[j]);
+      for (int j = 0; j < 8; ++j) sum += c[j];
+      int suf = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_down_sync(kFull, suf, o);
+        if (lane + o < 32) suf += y;
       }
-      const int inc = warp_inclusive_sum(s);
-      const int exc = inc - s;
-      if (exc < krem && inc >= krem) {
-        int acc = exc;
+      const int higher = suf - sum;  // members in the bins of higher lanes
+      if (higher < krem && suf >= krem) {
+        int acc = higher;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (acc + static_cast<int>(c[j]) >= krem) {
-            bc[0] = 255 - 8 * lane - j;
+        for (int j = 7; j >= 0; --j) {
+          if (acc + c[j] >= krem) {
+            bc[0] = 8 * lane + j;
             bc[1] = acc;
             break;
           }
-          acc += static_cast<int>(c[j]);
+          acc += c[j];
         }
       }
     }
