@@ -47,8 +47,12 @@ SYMBOLS = (
     "prr_version", "prr_status_string", "prr_workspace_bytes", "prr_workspace_init",
     "prr_get_device_status", "prr_append_kv", "prr_update_summaries", "prr_select_topk",
     "prr_ema_predict", "prr_speculate", "prr_repair_merge", "prr_decode_step",
-    "prr_decode_step_fused",
+    "prr_decode_step_fused", "prr_select_topk_static",
 )
+
+# mirrors PRR_SELECT_STATIC_MAX_BLOCKS / PRR_SELECT_STATIC_SCRATCH_BYTES in include/prr.h
+SELECT_STATIC_MAX_BLOCKS = 1 << 20
+SELECT_STATIC_SCRATCH_BYTES = 256 + 65536 * 4 + SELECT_STATIC_MAX_BLOCKS * 4
 
 STATUS = {0: "PRR_OK", 1: "PRR_ERR_INVALID_ARG", 2: "PRR_ERR_SHAPE", 3: "PRR_ERR_CAPACITY",
           4: "PRR_ERR_CUDA", 5: "PRR_ERR_DEVICE_STATUS", 6: "PRR_ERR_TIMEOUT"}
@@ -96,6 +100,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     L.prr_decode_step.argtypes = [dims, ctypes.POINTER(PrrStepBuffers), vp, sz, vp, vp,
                                   ctypes.POINTER(PrrStepEvents)]
     L.prr_decode_step_fused.argtypes = [dims, ctypes.POINTER(PrrStepBuffers), vp, sz, _i32, vp]
+    L.prr_select_topk_static.argtypes = [dims, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     for name in SYMBOLS:
         if name not in ("prr_version", "prr_status_string", "prr_workspace_bytes"):
             getattr(L, name).restype = ctypes.c_int
@@ -211,6 +216,14 @@ def prr_select_topk(dims, q, summ, seq_lens, pred, sel, missed, n_missed, keep, 
                                   _ptr(pred), _ptr(sel), _ptr(missed), _ptr(n_missed), _ptr(keep),
                                   _ptr(ws), _stream(stream)),
            "prr_select_topk")
+
+
+def prr_select_topk_static(dims, q, summ, seq_lens, pred, sel, missed, n_missed, keep,
+                           status=None, stream=None) -> None:
+    _check(load().prr_select_topk_static(ctypes.byref(_dims(dims)), _ptr(q), _ptr(summ), _ptr(seq_lens),
+                                         _ptr(pred), _ptr(sel), _ptr(missed), _ptr(n_missed),
+                                         _ptr(keep), _ptr(status), _stream(stream)),
+           "prr_select_topk_static")
 
 
 def prr_ema_predict(dims, ema, sel, seq_lens, pred_next, ws, stream=None) -> None:

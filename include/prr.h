@@ -242,6 +242,39 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* buf, vo
 prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* buf, void* ws,
                                  size_t ws_bytes, int32_t step_parity, cudaStream_t stream);
 
+/* Largest B*Hkv*ceil(cap_tokens/bs) that prr_select_topk_static accepts, and the bytes
+ * of device memory its fixed scratch array occupies on every GPU that loads the
+ * library (status word + 65536 chunk tickets + one 32-bit key per block). */
+#define PRR_SELECT_STATIC_MAX_BLOCKS (1 << 20)
+#define PRR_SELECT_STATIC_SCRATCH_BYTES (256 + 65536 * 4 + (size_t)PRR_SELECT_STATIC_MAX_BLOCKS * 4)
+
+/* prr_select_topk without a caller-supplied workspace, for callers that cannot
+ * allocate device memory: code running inside another runtime's memory pool with no
+ * access to its allocator, hosts that forbid cudaMalloc once serving has started
+ * (an allocation can synchronise the device or invalidate an ongoing stream capture),
+ * and deployments that fix every buffer at build time.  The paper has no counterpart:
+ * this is a packaging variant of the selection step, not a step of the method.
+ *
+ * Same arguments, results and shape rules as prr_select_topk, minus `ws`; the caller
+ * still passes every input and output.  The kernel's scratch (status word, per-unit
+ * chunk tickets, per-block score keys) lives in one fixed array inside the library,
+ * PRR_SELECT_STATIC_SCRATCH_BYTES per GPU, held from the moment the library's device
+ * code is loaded on that GPU until the process exits.
+ *   status: optional device int32; receives this call's device-side status code
+ *           (0 = ok, else one of PRR_DEV_*), written on `stream` after the kernel.
+ * Returns PRR_ERR_CAPACITY, without enqueuing anything, when
+ * B*Hkv*ceil(cap_tokens/bs) > PRR_SELECT_STATIC_MAX_BLOCKS.  Calls no cudaMalloc,
+ * cudaFree or other allocating routine.  The first call on each device (made with
+ * that device current) looks up the array's device address and keeps it; make that
+ * first call before any stream capture.  Every call clears the status word and the
+ * tickets on `stream` (the keys are always rewritten before use).  All calls share
+ * the one array: calls whose work may overlap on the GPU (different streams without
+ * ordering between them) race and give undefined results; order them on one stream. */
+prr_status prr_select_topk_static(const prr_dims* dims, const uint16_t* q, const uint16_t* summ,
+                                  const int32_t* seq_lens, const int32_t* pred, int32_t* sel,
+                                  int32_t* missed, int32_t* n_missed, uint8_t* keep,
+                                  int32_t* status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
