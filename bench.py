@@ -196,6 +196,21 @@ def recorded_traffic(kernel: str, workload: str):
     return None
 
 
+def reduce_over_ranks(tokens: float, seconds: float, e2e_value, world: int, device: str):
+    """Whole-job numbers of a replicas run: tokens summed over ranks, time = the max
+    over ranks (the slowest replica bounds the job), end-to-end throughput summed.
+    Every rank makes the same collective calls in the same order."""
+    if world <= 1:
+        return float(tokens), float(seconds), e2e_value
+    import torch
+    import torch.distributed as dist
+    v = torch.tensor([float(tokens), float(e2e_value or 0.0)], dtype=torch.float64, device=device)
+    m = torch.tensor([float(seconds)], dtype=torch.float64, device=device)
+    dist.all_reduce(v, op=dist.ReduceOp.SUM)
+    dist.all_reduce(m, op=dist.ReduceOp.MAX)
+    return v[0].item(), m[0].item(), (v[1].item() if e2e_value is not None else None)
+
+
 # ----------------------------------------------------------------------------- CPU oracle timing
 
 def oracle_run(w: W.Workload, warmup: int, steps: int, budget_s: float, nthreads: int):
@@ -463,17 +478,10 @@ def run_gpu(args):
             status = status or -1
 
     # ---------------- reduce over ranks
-    tot_tokens, max_time = tokens, my_time
-    if world > 1:
-        tt = torch.tensor([float(tokens)], device="cuda")
-        mt = torch.tensor([my_time], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.SUM)
-        dist.all_reduce(mt, op=dist.ReduceOp.MAX)
-        tot_tokens, max_time = tt.item(), mt.item()
-        if e2e is not None:
-            ev = torch.tensor([e2e["value"]], device="cuda")
-            dist.all_reduce(ev, op=dist.ReduceOp.SUM)
-            e2e["value"] = ev.item()
+    tot_tokens, max_time, e2e_total = reduce_over_ranks(tokens, my_time, e2e["value"] if e2e else None,
+                                                        world, "cuda")
+    if e2e is not None:
+        e2e["value"] = e2e_total
     value = tot_tokens / max_time
 
     # ---------------- roofline: the fused step kernel is the step's only kernel
