@@ -313,7 +313,8 @@ def run_gpu(args):
 
     e2e_steps = 0 if args.no_e2e else args.steps
     cmp_steps = 0 if args.no_streams else min(args.steps, 100)
-    total = 2 + args.warmup + args.steps + e2e_steps + 2 * cmp_steps + 8
+    n_levels = max(len(w.forced_overlaps or ()), 1)
+    total = 2 + args.warmup + n_levels * (args.steps + min(cmp_steps, 8)) + e2e_steps + 2 * cmp_steps + 8
     cap = w.N0 + total
     dims = Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, bs=w.bs, cap_tokens=cap, K=w.K, P=w.P, alpha=w.alpha)
     dec = PRRDecoder(dims)
@@ -335,10 +336,27 @@ def run_gpu(args):
         ev.record(main)
     t = 0
 
-    def prepare(step):
+    def prepare(step, flush_l2=True):
         dec.append(kn_d[step], vn_d[step], stream=main)
         dec.q.copy_(qs_d[step])
-        flush.zero_()
+        if flush_l2:
+            flush.zero_()
+
+    def force_prediction(step, overlap, level):
+        """Replace Pred_t by a set with a forced overlap with this step's true top-K.
+        S_t comes from the library (fold the appended key, then select); the forced set
+        is built on the host from the seeded generator.  Runs before the L2 flush."""
+        _abi.prr_update_summaries(dims, dec.k_cache, None, None, dec.seq_lens, 1, dec.summ, dec.ws, main)
+        _abi.prr_select_topk(dims, dec.q, dec.summ, dec.seq_lens, dec.pred, dec.sel, dec.missed,
+                             dec.n_missed, dec.keep, dec.ws, main)
+        sel = dec.sel.cpu().numpy()
+        nb = w.nb(w.N0 + step + 1)
+        ph = np.full((w.B, w.Hkv, max(w.P, 1)), -1, np.int32)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                fp = W.forced_prediction(w, sel[b, h][sel[b, h] >= 0], nb, overlap, level, step, b, h)
+                ph[b, h, :len(fp)] = fp[:w.P]
+        dec.pred.copy_(torch.from_numpy(ph))
 
     # eager warm-up of both implementations, then one graph per parity of each
     for fused in (True, False):
@@ -382,40 +400,79 @@ def run_gpu(args):
     torch.cuda.synchronize()
 
     # ---------------- timed region: fused single-launch step
+    # One pass over the levels: the EMA predictor's own sets, or (repair sweep) each
+    # forced overlap level in turn, args.steps timed steps per level.
+    levels = list(enumerate(w.forced_overlaps)) if w.forced_overlaps else [None]
     clocks = ClockSampler(f"GPU-{torch.cuda.get_device_properties(local).uuid}")
     clocks.wait_first()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     keep_sum = torch.zeros((), dtype=torch.int64, device="cuda")
     missed_sum = torch.zeros((), dtype=torch.int64, device="cuda")
     tokens = 0
-    step_bytes, timed_n = [], []
+    step_ms, step_bytes, timed_n, level_rows = [], [], [], []
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    for i in range(args.steps):
-        prepare(t)
-        starts[i].record(main)
-        replay("fused")
-        ends[i].record(main)
-        keep_sum += dec.keep.sum()
-        missed_sum += dec.n_missed.sum()
-        n = w.N0 + t + 1
-        timed_n.append(n)
-        tokens += w.B * n
-        step_bytes.append(algorithmic_bytes(w, n))
-        t += 1
-    torch.cuda.synchronize()
+    for lvl in levels:
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        lv_keep = torch.zeros((), dtype=torch.int64, device="cuda")
+        lv_missed = torch.zeros((), dtype=torch.int64, device="cuda")
+        for i in range(args.steps):
+            if lvl is None:
+                prepare(t)
+            else:
+                prepare(t, flush_l2=False)
+                force_prediction(t, lvl[1], lvl[0])
+                flush.zero_()
+            starts[i].record(main)
+            replay("fused")
+            ends[i].record(main)
+            lv_keep += dec.keep.sum()
+            lv_missed += dec.n_missed.sum()
+            n = w.N0 + t + 1
+            timed_n.append(n)
+            tokens += w.B * n
+            step_bytes.append(algorithmic_bytes(w, n))
+            t += 1
+        torch.cuda.synchronize()
+        lv_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+        step_ms += lv_ms
+        keep_sum += lv_keep
+        missed_sum += lv_missed
+        if lvl is not None:
+            keff = min(w.K, w.nb(w.N0))
+            row = {"overlap": lvl[1], "kept_blocks": W.forced_kept_count(lvl[1], keff),
+                   "us_per_step": statistics.mean(lv_ms) * 1e3, "us_per_step_p50": statistics.median(lv_ms) * 1e3,
+                   "predictor_overlap": lv_keep.item() / (args.steps * w.units * keff),
+                   "repaired_blocks_per_unit": lv_missed.item() / (args.steps * w.units)}
+            if cmp_steps:  # per-kernel times of the two-stream step at this level
+                kern, s_ms = {"select": [], "repair": [], "combine": [], "spec": [], "ema": []}, []
+                sa = torch.cuda.Event(enable_timing=True)
+                sb = torch.cuda.Event(enable_timing=True)
+                for _ in range(min(cmp_steps, 8)):
+                    prepare(t, flush_l2=False)
+                    force_prediction(t, lvl[1], lvl[0])
+                    flush.zero_()
+                    sa.record(main)
+                    replay("streams")
+                    sb.record(main)
+                    main.synchronize()
+                    s_ms.append(sa.elapsed_time(sb))
+                    for name, dur in kernel_spans(marks).items():
+                        kern[name].append(dur)
+                    t += 1
+                row["streams_us_per_step"] = statistics.mean(s_ms) * 1e3
+                row["streams_kernels_us"] = {k: statistics.mean(v) * 1e3 for k, v in kern.items()}
+            level_rows.append(row)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     my_time = sum(step_ms) / 1e3
     status = dec.device_status()
 
     # ---------------- two-stream implementation on the same trajectory (per-kernel marks)
     streams = None
-    if cmp_steps:
+    if cmp_steps and not w.forced_overlaps:
         kern = {"select": [], "repair": [], "combine": [], "ema": [], "spec": []}
         s_ms, overlap_frac = [], []
         sa = torch.cuda.Event(enable_timing=True)
@@ -486,13 +543,14 @@ def run_gpu(args):
 
     # ---------------- roofline: the fused step kernel is the step's only kernel
     keff = min(w.K, w.nb(w.N0))
-    overlap = keep_sum.item() / (args.steps * w.units * keff) if w.P > 0 else 0.0
+    n_timed = len(step_ms)
+    overlap = keep_sum.item() / (n_timed * w.units * keff) if w.P > 0 else 0.0
     step_algo = statistics.mean(b["total"] for b in step_bytes)
     step_mean_ms = statistics.mean(step_ms)
     achieved = step_algo / (step_mean_ms * 1e-3) / 1e9
     traffic = recorded_traffic("fused_step_kernel", w.name)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": n_timed,
         "warmup": args.warmup, "ms_per_step": step_mean_ms, "us_per_step": step_mean_ms * 1e3,
         "us_per_step_p50": statistics.median(step_ms) * 1e3,
         "us_per_step_p90": float(np.percentile(step_ms, 90)) * 1e3,
@@ -505,9 +563,10 @@ def run_gpu(args):
         "step_roofline": {"algorithmic_bytes_per_step": step_algo, "achieved_gbs": achieved,
                           "frac_of_8tbs": achieved / NOMINAL_HBM_GBS, "frac_of_measured": achieved / hbm_peak},
         "predictor_overlap": overlap,
-        "repaired_blocks_per_unit": missed_sum.item() / (args.steps * w.units),
+        "repaired_blocks_per_unit": missed_sum.item() / (n_timed * w.units),
+        "repair_sweep": level_rows or None,
         "streams_path": streams,
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": n_timed,
         "clocks": clk, "device_status": status,
     }
     if rank == 0:

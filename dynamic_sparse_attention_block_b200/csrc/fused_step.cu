@@ -1,14 +1,17 @@
 // fused_step.cu -- the whole PRR decode step in ONE persistent launch.
 //
 // Resident CTAs (128 threads) take work items from one atomic counter, in this order:
-//   1. SEL     (unit, chunk of 128 blocks): tail-summary fold, block scores -> keys; the
-//              last chunk of a unit runs the top-K finisher and publishes S_t.
-//   2. SPEC    (unit, predicted slot): speculative partial of block Pred_t[slot].  A
+//   1. SEL     (unit, chunk of 32-128 blocks): tail-summary fold, block scores -> keys.
+//   2. FIN     (unit): once the unit's chunks are scored, the top-K finisher; publishes
+//              S_t, the missed set and the keep mask.
+//   3. EMA     (unit): predictor update with S_t and Pred_{t+1}; starts copying its
+//              state at once and waits for S_t, then runs while speculation streams.
+//   4. SPEC    (unit, predicted slot): speculative partial of block Pred_t[slot].  A
 //              speculative item that starts after its unit's selection is published
 //              skips a block that selection dropped (its partial would be discarded).
-//   3. REPAIR  (unit, missed slot): partial of a missed block (waits for S_t).
-//   4. EMA     (unit): predictor update with S_t and Pred_{t+1} (waits for S_t).
-//   5. COMBINE (unit, query head): LSE merge of kept + repaired partials (waits for all
+//   5. REPAIR  (unit, r < R): partials of the missed blocks in slots r, r + R, ...
+//              (waits for S_t).
+//   6. COMBINE (unit, query head): LSE merge of kept + repaired partials (waits for all
 //              of the unit's speculative and repair partials).
 // This is the PRR runtime (abstract; method summary; contributions (1)-(3)) scheduled
 // for a 148-SM part: speculation overlaps selection inside the launch, selection work
@@ -28,24 +31,34 @@
 
 namespace prr {
 
-constexpr int kFusedChunk = 128;  // blocks per SEL item (4 warps x 32 rows)
+constexpr int kFusedChunk = 128;  // most blocks per SEL item (4 warps x 32 rows)
+
+// Blocks per SEL item: a multiple of 32 in [32, 128], about units*maxnb/512, so that a
+// short context still spreads its scan over many CTAs and a long one moves 64 KB per item.
+__host__ __device__ inline int fused_chunk_blocks(int units, int maxnb) {
+  long long c = (static_cast<long long>(units) * maxnb + 511) / 512;
+  c = ((c + 31) / 32) * 32;
+  return static_cast<int>(c < 32 ? 32 : (c > kFusedChunk ? kFusedChunk : c));
+}
 
 struct FusedCtl {
   unsigned* work;        // next item
   unsigned* abort;       // set on a timed-out wait
   unsigned* sel_loaded;  // SEL items whose summary tile has landed
   unsigned* sel_finished;  // units whose S_t is published
-  unsigned* sel_cnt;     // [units] finished SEL chunks
-  unsigned* sel_done;    // [units] S_t published
+  unsigned* sel_cnt;     // [units] scored SEL chunks
+  unsigned* sel_done;    // [units] 0, then 1 + |M_t| once S_t is published
   unsigned* p_act;       // [units] active speculative slots (published with S_t)
   unsigned* spec_done;   // [units] finished (or skipped) speculative items
   unsigned* rep_done;    // [units] finished repair items
+  unsigned* keepf;       // [units][P] 0 until S_t is known, then 1 | keep << 1
 };
 
 __device__ __forceinline__ FusedCtl ctl_view(const Params& p, int parity) {
   unsigned* b = p.ctl + static_cast<size_t>(parity) * p.ctl_words;
   const int U = p.units;
-  return FusedCtl{b, b + 1, b + 2, b + 3, b + 16, b + 16 + U, b + 16 + 2 * U, b + 16 + 3 * U, b + 16 + 4 * U};
+  return FusedCtl{b,          b + 1,          b + 2,          b + 3,         b + 16,
+                  b + 16 + U, b + 16 + 2 * U, b + 16 + 3 * U, b + 16 + 4 * U, b + 16 + 5 * U};
 }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -54,14 +67,18 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   return v;
 }
 
-// CTA-wide bounded wait until *flag >= target.  Thread 0 polls; the verdict is shared.
-__device__ bool wait_geq(const unsigned* flag, unsigned target, const FusedCtl& C, int* status, int* sh) {
+// CTA-wide bounded wait until *flag >= target.  Thread 0 polls; the verdict is shared,
+// and every thread gets the flag value thread 0 saw last in *seen (if given).
+__device__ bool wait_geq(const unsigned* flag, unsigned target, const FusedCtl& C, int* status, int* sh,
+                         unsigned* seen = nullptr) {
   if (threadIdx.x == 0) {
     int ok = 1;
-    if (ld_acquire(flag) < target) {
+    unsigned v = ld_acquire(flag);
+    if (v < target) {
       const uint64_t t0 = global_ns();
       for (;;) {
-        if (ld_acquire(flag) >= target) break;
+        v = ld_acquire(flag);
+        if (v >= target) break;
         if (ld_acquire(C.abort)) {
           ok = 0;
           break;
@@ -76,17 +93,20 @@ __device__ bool wait_geq(const unsigned* flag, unsigned target, const FusedCtl& 
       }
     }
     sh[0] = ok;
+    sh[4] = static_cast<int>(v);
   }
   __syncthreads();
   const bool ok = sh[0] != 0;
+  if (seen) *seen = static_cast<unsigned>(sh[4]);
   __syncthreads();
   return ok;
 }
 
+// Signal that this CTA's item is complete: the barrier orders every thread's writes
+// before thread 0's release, which a consumer pairs with an acquire load of the counter.
 __device__ __forceinline__ void count_done(unsigned* counter) {
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) atomicAdd(counter, 1u);
+  if (threadIdx.x == 0) red_release_add(counter, 1u);
 }
 
 template <int D>
@@ -105,31 +125,34 @@ struct FusedSel {
 // ---------------------------------------------------------------- SEL item
 template <int D>
 __device__ void sel_item(const Params& p, const FusedCtl& C, int u, int chunk, unsigned char* smem, uint64_t* bar,
-                         uint32_t& ph, int* sh) {
+                         uint32_t& ph) {
   using L = FusedSel<D>;
   constexpr int ROWB = L::ROWB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c0 = chunk * p.fchunk_blocks;
+  uint16_t* summ_unit = p.summ + static_cast<size_t>(u) * p.maxnb * 2 * D;
+  // The copy covers the chunk's rows up to the allocation (not the sequence length), so
+  // it starts before seq_lens has been read; rows past the last block are never used.
+  const int alloc_rows = max(0, min(p.fchunk_blocks, p.maxnb - c0));
+  if (tid == 0 && alloc_rows > 0) {
+    fence_proxy_async();
+    mbar_expect_tx(bar, static_cast<uint32_t>(alloc_rows) * ROWB);
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(summ_unit) + static_cast<size_t>(c0) * ROWB;
+    for (int w = 0; w < 4; ++w) {
+      const int rows = min(32, alloc_rows - 32 * w);
+      if (rows > 0) bulk_load(smem + w * 32 * ROWB, src + static_cast<size_t>(w) * 32 * ROWB, rows * ROWB, bar);
+    }
+  }
   const int n = checked_len(p, u / p.Hkv);
   const int nb = (n + p.bs - 1) / p.bs;
-  const int c0 = chunk * kFusedChunk;
-  const int cnt = max(0, min(kFusedChunk, nb - c0));
+  const int cnt = max(0, min(p.fchunk_blocks, nb - c0));
   const int tail = n > 0 ? (n - 1) / p.bs : -1;
   const bool own_tail = p.append_summary && tail >= c0 && tail < c0 + cnt;
-  uint16_t* summ_unit = p.summ + static_cast<size_t>(u) * p.maxnb * 2 * D;
   const size_t aux = L::aux(p.maxnb);
   float4* coef_lo = reinterpret_cast<float4*>(smem + aux);
   float4* coef_hi = coef_lo + L::C;
   uint16_t* newk = reinterpret_cast<uint16_t*>(coef_hi + L::C);
 
-  if (tid == 0 && cnt > 0) {
-    fence_proxy_async();
-    mbar_expect_tx(bar, static_cast<uint32_t>(cnt) * ROWB);
-    const unsigned char* src = reinterpret_cast<const unsigned char*>(summ_unit) + static_cast<size_t>(c0) * ROWB;
-    for (int w = 0; w < 4; ++w) {
-      const int rows = min(32, cnt - 32 * w);
-      if (rows > 0) bulk_load(smem + w * 32 * ROWB, src + static_cast<size_t>(w) * 32 * ROWB, rows * ROWB, bar);
-    }
-  }
   load_group_coef<D>(p, u, coef_lo, coef_hi);
   if (own_tail) {
     const uint16_t* krow = p.kc + (static_cast<size_t>(u) * p.cap + (n - 1)) * D;
@@ -137,7 +160,7 @@ __device__ void sel_item(const Params& p, const FusedCtl& C, int u, int chunk, u
       reinterpret_cast<uint4*>(newk)[c] = __ldg(reinterpret_cast<const uint4*>(krow) + c);
   }
   __syncthreads();
-  if (cnt > 0) {
+  if (alloc_rows > 0) {
     const bool ok = __syncthreads_and(mbar_wait(bar, ph, p.status));
     ph ^= 1u;
     if (!ok) {
@@ -153,37 +176,67 @@ __device__ void sel_item(const Params& p, const FusedCtl& C, int u, int chunk, u
     if (own_tail && tail >= first && tail < first + rows)
       fold_tail_row<D>(reinterpret_cast<uint32_t*>(tile + (tail - first) * ROWB), newk, ((n - 1) % p.bs) == 0,
                        reinterpret_cast<uint32_t*>(summ_unit + static_cast<size_t>(tail) * 2 * D), lane);
-    if (lane < rows)
-      p.keys[static_cast<size_t>(u) * p.maxnb + first + lane] =
-          orderable(score_summary_row<D>(tile + lane * ROWB, coef_lo, coef_hi, lane));
+    uint32_t key = 0u;
+    if (lane < rows) {
+      key = orderable(score_summary_row<D>(tile + lane * ROWB, coef_lo, coef_hi, lane));
+      p.keys[static_cast<size_t>(u) * p.maxnb + first + lane] = key;
+    }
+    write_group_summary(p, u, first / 32, key, lane < rows);
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) sh[1] = (atomicAdd(C.sel_cnt + u, 1u) == static_cast<unsigned>(p.fchunks - 1)) ? 1 : 0;
-  __syncthreads();
-  if (!sh[1]) return;
-  __threadfence();
-  const FinishOut f = select_finish(p, u, nb, smem);  // tiles are dead: scratch at 0
-  __threadfence();  // every thread's outputs are visible before S_t is published
-  __syncthreads();
-  if (tid == 0) {
+  count_done(C.sel_cnt + u);  // the unit's FIN item waits for all its chunks
+}
+
+// ---------------------------------------------------------------- FIN item
+__device__ void fin_item(const Params& p, const FusedCtl& C, int u, unsigned char* smem, int* sh) {
+  if (!wait_geq(C.sel_cnt + u, static_cast<unsigned>(p.fchunks), C, p.status, sh)) return;
+  const int n = checked_len(p, u / p.Hkv);
+  const int nb = (n + p.bs - 1) / p.bs;
+  const FinishOut f = select_finish(p, u, nb, smem, C.keepf + static_cast<size_t>(u) * p.P);
+  __syncthreads();  // every thread's outputs precede the release below
+  if (threadIdx.x == 0) {
     C.p_act[u] = static_cast<unsigned>(f.p_active);
-    __threadfence();
-    atomicExch(C.sel_done + u, 1u);
-    atomicAdd(C.sel_finished, 1u);
+    st_release(C.sel_done + u, 1u + static_cast<unsigned>(f.n_missed));
+    red_release_add(C.sel_finished, 1u);
+  }
+}
+
+// ---------------------------------------------------------------- L2 prefetch
+// Items are handed out roughly round-robin, so item it + gridDim.x is about one round
+// ahead.  Asking L2 for its data now keeps HBM busy while CTAs compute; every byte is
+// still read once from HBM (the item later finds it in L2).  Only SEL and SPEC items
+// have addresses known before the launch ends selection.
+template <int D, int BS>
+__device__ __forceinline__ void prefetch_item(const Params& p, int ahead, int n_sel, int spec0, int n_spec) {
+  if (ahead < n_sel) {
+    const int u = ahead / p.fchunks, c0 = (ahead % p.fchunks) * p.fchunk_blocks;
+    const int rows = min(p.fchunk_blocks, p.maxnb - c0);
+    if (rows > 0)
+      prefetch_l2(p.summ + (static_cast<size_t>(u) * p.maxnb + c0) * 2 * D, static_cast<uint32_t>(rows) * 4 * D);
+  } else if (ahead >= spec0 && ahead < spec0 + n_spec) {
+    const int s = ahead - spec0, u = s / p.P, j = s % p.P;
+    const int blk = __ldg(p.pred + static_cast<size_t>(u) * p.P + j);  // read-only in this launch
+    if (blk >= 0 && blk < p.maxnb) {
+      const int t0 = blk * BS;
+      const int rows = min(BS, p.cap - t0);
+      if (rows > 0) {
+        const size_t off = (static_cast<size_t>(u) * p.cap + t0) * D;
+        prefetch_l2(p.kc + off, static_cast<uint32_t>(rows) * D * 2);
+        prefetch_l2(p.vc + off, static_cast<uint32_t>(rows) * D * 2);
+      }
+    }
   }
 }
 
 // ---------------------------------------------------------------- fused kernel
 template <int D, int BS>
-__global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(128, 3) fused_step_kernel(const __grid_constant__ CUtensorMap kmap,
                                                          const __grid_constant__ CUtensorMap vmap,
                                                          const __grid_constant__ Params p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.fused_region);  // K tile, V tile, summaries
-  int* sh = reinterpret_cast<int*>(bars + 3);                              // broadcast slots
+  int* sh = reinterpret_cast<int*>(bars + 3);                              // broadcast slots [8]
   const int tid = threadIdx.x;
   const FusedCtl C = ctl_view(p, p.parity);
 
@@ -201,12 +254,24 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
 
   uint32_t ph_attn = 0u, ph_sel = 0u;
   const int U = p.units;
-  const int n_sel = U * p.fchunks, n_spec = U * p.P, n_rep = U * p.K, n_ema = U;
+  const int R = p.rep_items;
+  const int n_sel = U * p.fchunks, n_fin = U, n_spec = U * p.P, n_ema = U, n_rep = U * R;
   const int n_comb = U * p.G;
-  const int total = n_sel + n_spec + n_rep + n_ema + n_comb;
+  const int total = n_sel + n_fin + n_spec + n_ema + n_rep + n_comb;
 
+  // SEL, SPEC and REPAIR items take their CTA's next ticket as they start (thread 0),
+  // so the streaming phases never wait for the work counter.  FIN, EMA and COMBINE
+  // items do not: a long finisher or wait must not hold back a ticket that an idle CTA
+  // could run.
+  // Still deadlock-free: the lowest unfinished item is always being processed, because
+  // a CTA holding a prefetched ticket is working on a lower item.
+  constexpr unsigned kNoTicket = 0xFFFFFFFFu;
+  unsigned next_ticket = kNoTicket;
   for (;;) {
-    if (tid == 0) sh[2] = static_cast<int>(atomicAdd(C.work, 1u));
+    if (tid == 0) {
+      sh[2] = static_cast<int>(next_ticket != kNoTicket ? next_ticket : atomicAdd(C.work, 1u));
+      next_ticket = kNoTicket;
+    }
     __syncthreads();
     int it = sh[2];
     __syncthreads();
@@ -220,15 +285,32 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
       p.trace[4 * static_cast<size_t>(it) + 3] = static_cast<unsigned long long>(it);
     }
     const int item_id = it;
+    if (tid == 32) prefetch_item<D, BS>(p, it + static_cast<int>(gridDim.x), n_sel, n_sel + n_fin + n_ema, n_spec);
 
     if (it < n_sel) {
-      sel_item<D>(p, C, it / p.fchunks, it % p.fchunks, smem, &bars[2], ph_sel, sh);
+      if (tid == 0) next_ticket = atomicAdd(C.work, 1u);
+      sel_item<D>(p, C, it / p.fchunks, it % p.fchunks, smem, &bars[2], ph_sel);
       __syncthreads();
       if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
       continue;
     }
     it -= n_sel;
+    if (it < n_fin) {
+      fin_item(p, C, it, smem, sh);
+      __syncthreads();
+      if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
+      continue;
+    }
+    it -= n_fin;
+    if (it < n_ema) {  // predictor for step t+1
+      ema_unit(p, it, smem, [&] { return wait_geq(C.sel_done + it, 1u, C, p.status, sh); });
+      __syncthreads();
+      if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
+      continue;
+    }
+    it -= n_ema;
     if (it < n_spec) {  // speculation
+      if (tid == 0) next_ticket = atomicAdd(C.work, 1u);
       const int u = it / p.P, j = it % p.P;
       const int n = checked_len(p, u / p.Hkv);
       const int nb = (n + BS - 1) / BS;
@@ -238,8 +320,7 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
         // every selection tile has landed; gate 2: until every unit's S_t is published.
         if (p.spec_gate == 1) wait_geq(C.sel_loaded, static_cast<unsigned>(n_sel), C, p.status, sh);
         if (p.spec_gate == 2) wait_geq(C.sel_finished, static_cast<unsigned>(U), C, p.status, sh);
-        if (tid == 0) sh[3] = (ld_acquire(C.sel_done + u) != 0u &&
-                               __ldcg(p.keep + static_cast<size_t>(u) * p.P + j) == 0) ? 1 : 0;
+        if (tid == 0) sh[3] = (__ldcg(C.keepf + static_cast<size_t>(u) * p.P + j) == 1u) ? 1 : 0;  // dropped
         __syncthreads();
         const bool skip = sh[3] != 0;
         if (!skip) {
@@ -258,10 +339,12 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
     }
     it -= n_spec;
     if (it < n_rep) {  // repair
-      const int u = it / p.K, i = it % p.K;
-      if (wait_geq(C.sel_done + u, 1u, C, p.status, sh)) {
-        const int nm = min(max(__ldcg(p.n_missed + u), 0), p.K);
-        if (i < nm) {
+      if (tid == 0) next_ticket = atomicAdd(C.work, 1u);
+      const int u = it / R, r = it % R;
+      unsigned flag = 0u;
+      if (wait_geq(C.sel_done + u, 1u, C, p.status, sh, &flag)) {
+        const int nm = min(static_cast<int>(flag) - 1, p.K);  // |M_t| came with the flag
+        for (int i = r; i < nm; i += R) {  // missed slots r, r + R, ...
           const int n = checked_len(p, u / p.Hkv);
           const int nb = (n + BS - 1) / BS;
           const int blk = __ldcg(p.missed + static_cast<size_t>(u) * p.K + i);
@@ -284,18 +367,12 @@ __global__ void __launch_bounds__(128) fused_step_kernel(const __grid_constant__
       continue;
     }
     it -= n_rep;
-    if (it < n_ema) {  // predictor for step t+1
-      if (wait_geq(C.sel_done + it, 1u, C, p.status, sh)) ema_unit(p, it, smem);
-      __syncthreads();
-      if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();
-      continue;
-    }
-    it -= n_ema;
     {  // LSE merge of (unit, head)
       const int u = it / p.G, h = it % p.G;
-      if (wait_geq(C.sel_done + u, 1u, C, p.status, sh)) {
+      unsigned flag = 0u;
+      if (wait_geq(C.sel_done + u, 1u, C, p.status, sh, &flag)) {
+        const unsigned nm = static_cast<unsigned>(min(static_cast<int>(flag) - 1, p.K));
         const unsigned pa = __ldcg(C.p_act + u);
-        const unsigned nm = static_cast<unsigned>(min(max(__ldcg(p.n_missed + u), 0), p.K));
         // fold the speculative partials as soon as they are all written, then the repairs
         if (wait_geq(C.spec_done + u, pa, C, p.status, sh))
           combine_head<D>(p, u, h, smem, [&] { return wait_geq(C.rep_done + u, nm, C, p.status, sh); });
@@ -320,7 +397,8 @@ static size_t fused_region_bytes(const Params& p) {
 template <int D, int BS>
 static cudaError_t launch_fused_t(Params p, const CUtensorMap& kmap, const CUtensorMap& vmap, cudaStream_t s,
                                   int priority, int sms, int* grid_out) {
-  p.fchunks = (p.maxnb + kFusedChunk - 1) / kFusedChunk;
+  p.fchunk_blocks = fused_chunk_blocks(p.units, p.maxnb);
+  p.fchunks = (p.maxnb + p.fchunk_blocks - 1) / p.fchunk_blocks;
   p.fused_region = static_cast<int>(fused_region_bytes<D, BS>(p));
   const size_t smem = 1024 + static_cast<size_t>(p.fused_region) + 3 * 8 + 8 * 4;
   const void* fn = reinterpret_cast<const void*>(fused_step_kernel<D, BS>);
@@ -330,7 +408,7 @@ static cudaError_t launch_fused_t(Params p, const CUtensorMap& kmap, const CUten
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_step_kernel<D, BS>, 128, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  const long long items = static_cast<long long>(p.units) * (p.fchunks + p.P + p.K + 1 + p.G);
+  const long long items = static_cast<long long>(p.units) * (p.fchunks + 1 + p.P + 1 + p.rep_items + p.G);
   long long grid = static_cast<long long>(per_sm) * sms;
   if (grid > items) grid = items;
   if (grid_out) *grid_out = static_cast<int>(grid);
@@ -350,7 +428,8 @@ cudaError_t launch_fused(const Params& p, const CUtensorMap& kmap, const CUtenso
 
 size_t fused_smem_bytes(const Params& p) {
   Params q = p;
-  q.fchunks = (q.maxnb + kFusedChunk - 1) / kFusedChunk;
+  q.fchunk_blocks = fused_chunk_blocks(q.units, q.maxnb);
+  q.fchunks = (q.maxnb + q.fchunk_blocks - 1) / q.fchunk_blocks;
   size_t r;
   if (p.d == 128) r = p.bs == 128 ? fused_region_bytes<128, 128>(q) : fused_region_bytes<128, 64>(q);
   else r = p.bs == 128 ? fused_region_bytes<64, 128>(q) : fused_region_bytes<64, 64>(q);

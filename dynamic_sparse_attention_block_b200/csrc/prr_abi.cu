@@ -3,6 +3,7 @@
 // orchestration of one decode step.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -48,6 +49,8 @@ WsLayout layout_for(const prr_dims* d) {
   off = align256(off + 4 * units);
   L.keys = off;
   off = align256(off + 4 * units * maxnb);
+  L.gsum = off;
+  off = align256(off + 8 * units * ((maxnb + 31) / 32));
   L.rm = off;
   off = align256(off + 4 * units * G * d->K);
   L.rl = off;
@@ -55,7 +58,7 @@ WsLayout layout_for(const prr_dims* d) {
   L.rO = off;
   off = align256(off + 4 * units * G * d->K * d->d);
   L.ctl = off;
-  off = align256(off + 4 * 2 * (16 + 5 * units));
+  off = align256(off + 4 * 2 * (16 + 5 * units + units * static_cast<size_t>(d->P)));
   L.total = off;
   return L;
 }
@@ -127,17 +130,21 @@ Params base_params(const prr_dims* d, void* ws) {
     p.status = reinterpret_cast<int*>(w + L.status);
     p.sel_cnt = reinterpret_cast<unsigned*>(w + L.sel_cnt);
     p.keys = reinterpret_cast<uint32_t*>(w + L.keys);
+    p.gsum = reinterpret_cast<uint2*>(w + L.gsum);
     p.rm = reinterpret_cast<float*>(w + L.rm);
     p.rl = reinterpret_cast<float*>(w + L.rl);
     p.rO = reinterpret_cast<float*>(w + L.rO);
     p.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
   }
-  p.ctl_words = 16 + 5 * p.units;
+  p.ctl_words = 16 + 5 * p.units + p.units * p.P;
+  // repair items per unit of the fused step: enough to spread a unit's misses over
+  // many CTAs, few enough that empty items (most units miss little) stay cheap
+  p.rep_items = std::min(p.K, std::max(4, (1024 + p.units - 1) / p.units));
   {
     static int gate = -1;  // PRR_SPEC_GATE in {0, 1, 2} overrides the speculation gate
     if (gate < 0) {
       const char* e = std::getenv("PRR_SPEC_GATE");
-      gate = (e && e[0] >= '0' && e[0] <= '2') ? e[0] - '0' : 1;
+      gate = (e && e[0] >= '0' && e[0] <= '2') ? e[0] - '0' : 0;
     }
     p.spec_gate = gate;
   }

@@ -25,10 +25,11 @@ struct WsLayout {
   size_t status;     // int32 status word
   size_t sel_cnt;    // uint32 [units] chunk tickets of the selection kernel
   size_t keys;       // uint32 [units][maxnb] order-preserving block-score keys
+  size_t gsum;       // uint32x2 [units][ceil(maxnb/32)] per 32-block group: max key, tie mask
   size_t rm;         // float [units*G][K] repair partial max (base-2 logits)
   size_t rl;         // float [units*G][K] repair partial sum
   size_t rO;         // float [units*G][K][d] repair partial numerator
-  size_t ctl;        // uint32 [2][16 + 5*units] control words of the fused step
+  size_t ctl;        // uint32 [2][16 + 5*units + units*P] control words of the fused step
   size_t total;
 };
 
@@ -45,7 +46,9 @@ struct Params {
   int parity;        // which copy of the control words this launch uses
   int ctl_words;     // words per copy
   int fchunks;       // SEL items per unit
+  int fchunk_blocks; // blocks per SEL item
   int fused_region;  // bytes of the per-CTA shared-memory union
+  int rep_items;     // REPAIR items per unit; item r repairs missed slots r, r + rep_items, ...
   int spec_gate;     // speculative items wait: 0 no, 1 selection tiles landed, 2 all S_t published
   // caller buffers (any may be null when the kernel does not use it)
   const uint16_t* q;        // [B][Hq][d] bf16
@@ -69,6 +72,7 @@ struct Params {
   int* status;
   unsigned* sel_cnt;
   uint32_t* keys;
+  uint2* gsum;               // null: the finisher derives group maxima from the keys
   float* rm;
   float* rl;
   float* rO;

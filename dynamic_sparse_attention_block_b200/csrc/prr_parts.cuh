@@ -63,11 +63,17 @@ __device__ __forceinline__ void load_group_coef(const Params& p, int u, float4* 
   float* hi = reinterpret_cast<float*>(hi4);
   const uint16_t* qg = p.q + static_cast<size_t>(u) * p.G * D;
   for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    uint16_t qv[8];  // G <= 8: every head's load in flight before the first is used
+#pragma unroll
+    for (int h = 0; h < 8; ++h) qv[h] = h < p.G ? __ldg(qg + h * D + c) : static_cast<uint16_t>(0);
     float neg = 0.f, pos = 0.f;
-    for (int h = 0; h < p.G; ++h) {
-      const float x = __uint_as_float(static_cast<uint32_t>(qg[h * D + c]) << 16);
-      neg += fminf(x, 0.f);
-      pos += fmaxf(x, 0.f);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if (h < p.G) {
+        const float x = __uint_as_float(static_cast<uint32_t>(qv[h]) << 16);
+        neg += fminf(x, 0.f);
+        pos += fmaxf(x, 0.f);
+      }
     }
     const int e0 = c, e1 = D + c;  // min part, max part
     ((e0 & 7) < 4 ? lo[(e0 >> 3) * 4 + (e0 & 3)] : hi[(e0 >> 3) * 4 + (e0 & 3)]) = neg;
@@ -124,8 +130,35 @@ __device__ __forceinline__ void fold_tail_row(uint32_t* row, const uint16_t* new
 // True selected set (PRR abstract): the K best blocks under (score desc, index asc),
 // written in ascending block order.  missed = S \ Pred ascending, keep[j] = [Pred_j in S]
 // (PRR method summary, contributions (2)-(3)).  A predicted slot is active iff
-// 0 <= Pred_j < nb.  Keys come from p.keys (written by this or other CTAs); the keys
-// and the predicted list are fetched together (one round trip).
+// 0 <= Pred_j < nb.
+//
+// S = {key > T} plus the lowest-index blocks with key == T, T the K_eff-th largest key.
+// Group summaries: each scoring warp writes, for its group of 32 blocks, the group's
+// largest key and the mask of the blocks holding it.  From those alone the finisher
+// sees whether at least K_eff blocks tie at the overall maximum; then T is that maximum
+// and S is the first K_eff set bits of the maximal groups' masks -- no key is loaded
+// (this is the usual case when every block's bound saturates).  Otherwise one warp
+// finds T bit by bit from the most significant bit that the smallest and largest keys
+// differ in: T keeps a bit when at least K_eff keys are >= the candidate value.  That
+// needs no CTA barrier per step.
+
+constexpr int kBitRegs = 32;  // keys per lane kept in registers by the bit search (nb <= 1024)
+
+// Start of the bit search: the bits that the smallest and largest keys share, lower
+// bits zero (every key is >= it).
+__device__ __forceinline__ uint32_t bit_search_start(uint32_t lo, uint32_t hi) {
+  if (lo == hi) return hi;
+  const int top = 31 - __clz(lo ^ hi);  // highest differing bit
+  return top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+}
+
+// One warp (all lanes): summary of the warp's group of 32 blocks (`valid` lanes).
+__device__ __forceinline__ void write_group_summary(const Params& p, int u, int group, uint32_t key, bool valid) {
+  if (!p.gsum) return;
+  const uint32_t mx = __reduce_max_sync(kFull, valid ? key : 0u);
+  const unsigned mask = __ballot_sync(kFull, valid && key == mx);
+  if ((threadIdx.x & 31) == 0) p.gsum[static_cast<size_t>(u) * ((p.maxnb + 31) / 32) + group] = make_uint2(mx, mask);
+}
 
 struct FinishOut {
   int p_active;  // active predicted slots
@@ -133,28 +166,43 @@ struct FinishOut {
 };
 
 __host__ __device__ constexpr size_t finish_scratch_bytes(int maxnb) {
-  return 256 * 4 + 128 * 4 + 16 * 4 + static_cast<size_t>(maxnb) * 4 + 3 * static_cast<size_t>((maxnb + 31) / 32) * 4;
+  return 256 * 4 + 128 * 4 + 16 * 4 + static_cast<size_t>((maxnb + 31) / 32) * 8 + static_cast<size_t>(maxnb) * 4 +
+         3 * static_cast<size_t>((maxnb + 31) / 32) * 4;
 }
 
-__device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsigned char* scratch) {
-  const int tid = threadIdx.x, warp = tid >> 5;
+// keepf (optional, [P]): per predicted slot, 1 | keep << 1 once S_t is known.
+__device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsigned char* scratch,
+                                          unsigned* keepf = nullptr) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, NT = blockDim.x;
   const int W = (p.maxnb + 31) / 32;
-  unsigned* hist = reinterpret_cast<unsigned*>(scratch);  // 16-byte aligned
-  int* spred = reinterpret_cast<int*>(hist + 256);        // [128]
-  int* misc = spred + 128;                                // bc[2], counts
-  uint32_t* skeys = reinterpret_cast<uint32_t*>(misc + 16);
+  int* spred = reinterpret_cast<int*>(scratch + 256 * 4);  // [128]
+  int* misc = spred + 128;                                 // counts, T, n_gt
+  uint2* gs = reinterpret_cast<uint2*>(misc + 16);         // [W] group summaries
+  uint32_t* skeys = reinterpret_cast<uint32_t*>(gs + W);
   unsigned* bm_pred = skeys + p.maxnb;
   unsigned* bm_sel = bm_pred + W;
   unsigned* bm_eq = bm_sel + W;
+  const int Wn = (nb + 31) / 32;
 
   PRR_PHASE(0, u, 0);
-  for (int j = tid; j < p.P; j += blockDim.x) spred[j] = p.pred[static_cast<size_t>(u) * p.P + j];
-  load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb);
-  for (int i = tid; i < W; i += blockDim.x) bm_pred[i] = 0u;
+  const int keff = min(p.K, nb);
+  const bool take_all = keff >= nb;
+  const bool use_gs = p.gsum != nullptr && !take_all && keff > 0;
+  bool have_keys = false;
+  for (int j = tid; j < p.P; j += NT) spred[j] = p.pred[static_cast<size_t>(u) * p.P + j];
+  if (use_gs) {
+    const uint2* src = p.gsum + static_cast<size_t>(u) * W;
+    for (int g = tid; g < Wn; g += NT) gs[g] = __ldcg(src + g);
+  } else if (!take_all) {
+    load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb);
+    have_keys = true;
+  }
+  for (int i = tid; i < W; i += NT) bm_pred[i] = 0u;
+  if (tid < 16) misc[tid] = 0;
   __syncthreads();
   PRR_PHASE(0, u, 1);
   int active_local = 0;
-  for (int j = tid; j < p.P; j += blockDim.x) {
+  for (int j = tid; j < p.P; j += NT) {
     const int pv = spred[j];
     if (pv >= 0 && pv < nb) {
       ++active_local;
@@ -164,26 +212,151 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
       report(p.status, kDevBadPred);
     }
   }
-  const int keff = min(p.K, nb);
   uint32_t T = 0u;
   int n_gt = 0;
-  const bool take_all = keff >= nb;
-  if (keff > 0 && !take_all)
-    T = radix_kth_largest(
-        nb, keff, [&](int i) { return skeys[i]; }, [&](int) { return true; }, hist, misc, &n_gt);
+  bool tie_masks = false;  // S comes straight from the group tie masks
+  if (!take_all && keff > 0) {
+    unsigned* ms = reinterpret_cast<unsigned*>(misc);
+    // largest key and the number of blocks holding it
+    uint32_t mx = 0u;
+    if (use_gs) {
+      for (int g = tid; g < Wn; g += NT) mx = max(mx, gs[g].x);
+    } else {
+      for (int i = tid; i < nb; i += NT) mx = max(mx, skeys[i]);
+    }
+    mx = __reduce_max_sync(kFull, mx);
+    if (lane == 0) atomicMax(&ms[6], mx);
+    __syncthreads();
+    const uint32_t gmax = ms[6];
+    int ce = 0;
+    if (use_gs) {
+      for (int g = tid; g < Wn; g += NT) ce += gs[g].x == gmax ? __popc(gs[g].y) : 0;
+    } else {
+      for (int i = tid; i < nb; i += NT) ce += skeys[i] == gmax ? 1 : 0;
+    }
+    ce = __reduce_add_sync(kFull, ce);
+    if (lane == 0 && ce) atomicAdd(&misc[7], ce);
+    __syncthreads();
+    if (misc[7] >= keff) {
+      T = gmax;
+      tie_masks = use_gs;
+    } else {
+      if (!have_keys) {
+        load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb);
+        have_keys = true;
+        __syncthreads();
+      }
+      if (warp == 0) {  // T bit by bit; every candidate count is one warp reduction
+        uint32_t t, gt;
+        if (nb <= 32 * kBitRegs) {
+          // keys held in registers (padding 0 is below every candidate, which is > 0)
+          uint32_t kr[kBitRegs];
+#pragma unroll
+          for (int q = 0; q < kBitRegs; ++q) {
+            const int i = q * 32 + lane;
+            kr[q] = i < nb ? skeys[i] : 0u;
+          }
+          uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+          for (int q = 0; q < kBitRegs; ++q) {
+            if (q * 32 + lane < nb) lo = min(lo, kr[q]);
+            hi = max(hi, kr[q]);
+          }
+          lo = __reduce_min_sync(kFull, lo);
+          hi = __reduce_max_sync(kFull, hi);
+          t = bit_search_start(lo, hi);
+          if (lo != hi) {
+            for (int bit = 31 - __clz(lo ^ hi); bit >= 0; --bit) {
+              const uint32_t c = t | (1u << bit);
+              int cnt = 0;
+#pragma unroll
+              for (int q = 0; q < kBitRegs; ++q) cnt += kr[q] >= c ? 1 : 0;
+              if (__reduce_add_sync(kFull, cnt) >= static_cast<unsigned>(keff)) t = c;
+            }
+          }
+          int g = 0;
+#pragma unroll
+          for (int q = 0; q < kBitRegs; ++q) g += kr[q] > t ? 1 : 0;
+          gt = __reduce_add_sync(kFull, g);
+        } else {
+          uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+          for (int i = lane; i < nb; i += 32) {
+            lo = min(lo, skeys[i]);
+            hi = max(hi, skeys[i]);
+          }
+          lo = __reduce_min_sync(kFull, lo);
+          hi = __reduce_max_sync(kFull, hi);
+          t = bit_search_start(lo, hi);
+          if (lo != hi) {
+            for (int bit = 31 - __clz(lo ^ hi); bit >= 0; --bit) {
+              const uint32_t c = t | (1u << bit);
+              int cnt = 0;
+#pragma unroll 8
+              for (int i = lane; i < nb; i += 32) cnt += skeys[i] >= c ? 1 : 0;
+              if (__reduce_add_sync(kFull, cnt) >= static_cast<unsigned>(keff)) t = c;
+            }
+          }
+          int g = 0;
+          for (int i = lane; i < nb; i += 32) g += skeys[i] > t ? 1 : 0;
+          gt = __reduce_add_sync(kFull, g);
+        }
+        if (lane == 0) {
+          ms[8] = t;
+          misc[9] = static_cast<int>(gt);
+        }
+      }
+      __syncthreads();
+      T = ms[8];
+      n_gt = misc[9];
+    }
+  }
   PRR_PHASE(0, u, 2);
-  select_bitmap(
-      nb, take_all ? 0 : keff - n_gt,
-      [&](int i) {
-        if (take_all) return 1;
-        const uint32_t kv = skeys[i];
-        return kv > T ? 1 : (kv == T ? 0 : -1);
-      },
-      bm_sel, bm_eq);
   PRR_PHASE(0, u, 3);
+  if (tie_masks) {
+    // the first K_eff tied blocks in index order: trim the maximal groups' masks
+    if (warp == 0) {
+      int base = 0;
+      for (int w0 = 0; w0 < Wn; w0 += 32) {
+        const int wd = w0 + lane;
+        unsigned m = 0u;
+        if (wd < Wn) {
+          const uint2 g = gs[wd];
+          m = g.x == T ? g.y : 0u;
+        }
+        const int c = __popc(m);
+        const int inc = warp_inclusive_sum(c);
+        const int exc = base + inc - c;
+        unsigned keepm = 0u;
+        if (exc < keff) {
+          const int need = keff - exc;
+          keepm = m;
+          if (need < c) {
+            keepm = 0u;
+            unsigned e = m;
+            for (int r = 0; r < need; ++r) {
+              const unsigned low = e & (0u - e);
+              keepm |= low;
+              e ^= low;
+            }
+          }
+        }
+        if (wd < Wn) bm_sel[wd] = keepm;
+        base += __shfl_sync(kFull, inc, 31);
+      }
+    }
+    __syncthreads();
+  } else {
+    select_bitmap(
+        nb, take_all ? 0 : keff - n_gt,
+        [&](int i) {
+          if (take_all) return 1;
+          const uint32_t kv = skeys[i];
+          return kv > T ? 1 : (kv == T ? 0 : -1);
+        },
+        bm_sel, bm_eq);
+  }
   // three warps in parallel: selected list, missed list, keep mask
   int nm = 0;
-  const int Wn = (nb + 31) / 32;
   if (warp == 0) {
     warp_emit_bitmap(bm_sel, nullptr, Wn, p.sel + static_cast<size_t>(u) * p.K, p.K);
   } else if (warp == 1) {
@@ -193,10 +366,11 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
       misc[2] = nm;
     }
   }
-  for (int j = tid; j < p.P; j += blockDim.x) {
+  for (int j = tid; j < p.P; j += NT) {
     const int pv = spred[j];
-    p.keep[static_cast<size_t>(u) * p.P + j] =
-        (pv >= 0 && pv < nb && ((bm_sel[pv >> 5] >> (pv & 31)) & 1u)) ? 1 : 0;
+    const unsigned kv = (pv >= 0 && pv < nb && ((bm_sel[pv >> 5] >> (pv & 31)) & 1u)) ? 1u : 0u;
+    p.keep[static_cast<size_t>(u) * p.P + j] = static_cast<uint8_t>(kv);
+    if (keepf) keepf[j] = 1u | (kv << 1);
   }
   // active predicted slots (CTA sum of the per-thread counts)
   if (tid == 0) misc[3] = 0;
@@ -216,104 +390,153 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
 // in fp64 with separately rounded multiplies and add (no fused multiply-add), so the
 // state and the predicted set are bit-exact against the fp64 CPU oracle.
 // Pred_{t+1} = the min(P, nb) best blocks under (e desc, index asc), ascending, -1
-// beyond.  e >= 0, so its IEEE bit pattern orders like its value: the P-th largest
-// pattern is found by radix selection on the high word, then (unless the tied entries
-// agree on the low word) on the low word among entries tied on the high word; exact
-// ties go to the lowest block indices.
+// beyond.  e >= 0, so its IEEE bit pattern orders like its value.
+//
+// Candidate filter (exact): after the update every block of S_t holds e >= beta (a
+// rounded sum of beta and a non-negative term), so when P_eff <= |S_t| the P-th
+// largest e is >= beta and the whole predicted set lies among the blocks with
+// e >= beta.  Those candidates (typically about K of them, given temporal locality)
+// are collected during the update and ranked by counting: rank(i) = #{j : e_j > e_i,
+// or e_j == e_i and j < i}; rank < P_eff is selected.  Otherwise (P > |S_t|, no
+// update, or too many candidates) the general path runs: radix selection on the
+// high word, then on the low word among the entries tied on the high word.
+
+constexpr int kEmaCand = 512;  // candidates ranked by counting; more take the radix path
 
 __host__ __device__ constexpr size_t ema_scratch_bytes(int maxnb) {
-  return 256 * 4 + 16 * 4 + static_cast<size_t>(maxnb) * 8 + 3 * static_cast<size_t>((maxnb + 31) / 32) * 4;
+  return 256 * 4 + 16 * 4 + static_cast<size_t>(kEmaCand) * 12 + static_cast<size_t>(maxnb) * 8 +
+         3 * static_cast<size_t>((maxnb + 31) / 32) * 4;
 }
 
-__device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch) {
+// Every thread of the CTA calls it.  wait_sel() (CTA-wide) returns once S_t may be read,
+// false to give up; the state copy is started before it, so its latency is hidden.
+template <typename WaitFn>
+__device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, WaitFn wait_sel) {
   const int W = (p.maxnb + 31) / 32;
   unsigned* hist = reinterpret_cast<unsigned*>(scratch);  // 16-byte aligned
-  int* misc = reinterpret_cast<int*>(hist + 256);
-  uint32_t* hi = reinterpret_cast<uint32_t*>(misc + 16);
-  uint32_t* lo = hi + p.maxnb;
-  unsigned* bm = lo + p.maxnb;  // selected blocks of this step
-  unsigned* bsel = bm + W;      // predicted set
+  int* misc = reinterpret_cast<int*>(hist + 256);         // [4] candidates, [5] |S_t|
+  unsigned long long* ckey = reinterpret_cast<unsigned long long*>(misc + 16);
+  int* cidx = reinterpret_cast<int*>(ckey + kEmaCand);
+  double* ev = reinterpret_cast<double*>(cidx + kEmaCand);  // state, up to the allocation
+  unsigned* bm = reinterpret_cast<unsigned*>(ev + p.maxnb);  // selected blocks of this step
+  unsigned* bsel = bm + W;                                    // predicted set
   unsigned* beq = bsel + W;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   PRR_PHASE(1, u, 0);
-  const int n = checked_len(p, u / p.Hkv);
-  const int nb = (n + p.bs - 1) / p.bs;
   double* e = p.ema + static_cast<size_t>(u) * p.maxnb;
   const bool update = p.sel != nullptr;
-
-  // fetch the state and S_t together (many loads in flight per thread)
+  // state copy up to the allocation (entries >= nb are unused), before any wait
+  for (int i = tid; i < p.maxnb; i += blockDim.x) cp_async_8(ev + i, e + i);
+  for (int i = tid; i < W; i += blockDim.x) {
+    bm[i] = 0u;
+    bsel[i] = 0u;
+  }
+  if (tid == 0) {
+    misc[4] = 0;
+    misc[5] = 0;
+  }
+  if (!wait_sel()) {
+    cp_async_wait_all();
+    __syncthreads();
+    return;
+  }
   int sv = -1;
   if (update && tid < p.K) sv = __ldcg(p.sel + static_cast<size_t>(u) * p.K + tid);
-  for (int base = 0; base < nb; base += kBatch * static_cast<int>(blockDim.x)) {
-    double v[kBatch];
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const int i = base + q * blockDim.x + tid;
-      v[q] = i < nb ? e[i] : 0.0;
-    }
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const int i = base + q * blockDim.x + tid;
-      if (i < nb) {
-        const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(v[q]));
-        hi[i] = static_cast<uint32_t>(bits >> 32);
-        lo[i] = static_cast<uint32_t>(bits);
-      }
-    }
-  }
-  for (int i = tid; i < W; i += blockDim.x) bm[i] = 0u;
+  const int n = checked_len(p, u / p.Hkv);
+  const int nb = (n + p.bs - 1) / p.bs;
+  const int Wn = (nb + 31) / 32;
+  const int peff = min(p.P, nb);
+  cp_async_wait_all();
   __syncthreads();
+  bool ranked = false;
   if (update) {
     for (int i = tid; i < p.K; i += blockDim.x) {
       const int v = i == tid ? sv : __ldcg(p.sel + static_cast<size_t>(u) * p.K + i);
       if (v >= 0 && v < nb) atomicOr(&bm[v >> 5], 1u << (v & 31));
     }
     __syncthreads();
+    int nsel = 0;
+    for (int i = tid; i < Wn; i += blockDim.x) nsel += __popc(bm[i]);
+    if (nsel) atomicAdd(&misc[5], nsel);
+    __syncthreads();
+    const bool filter = peff > 0 && peff < nb && peff <= misc[5];
     const double alpha = p.alpha;
     const double beta = __dsub_rn(1.0, alpha);
-    for (int i = tid; i < nb; i += blockDim.x) {
-      const double x0 = __longlong_as_double(static_cast<long long>((static_cast<unsigned long long>(hi[i]) << 32) | lo[i]));
-      const double ind = ((bm[i >> 5] >> (i & 31)) & 1u) ? 1.0 : 0.0;
-      const double x = __dadd_rn(__dmul_rn(alpha, x0), __dmul_rn(beta, ind));
-      e[i] = x;
-      const unsigned long long bits = static_cast<unsigned long long>(__double_as_longlong(x));
-      hi[i] = static_cast<uint32_t>(bits >> 32);
-      lo[i] = static_cast<uint32_t>(bits);
+    for (int base = 0; base < nb; base += blockDim.x) {  // warp-uniform trip count
+      const int i = base + tid;
+      bool cand = false;
+      unsigned long long bits = 0ull;
+      if (i < nb) {
+        const double ind = ((bm[i >> 5] >> (i & 31)) & 1u) ? 1.0 : 0.0;
+        const double x = __dadd_rn(__dmul_rn(alpha, ev[i]), __dmul_rn(beta, ind));
+        e[i] = x;
+        ev[i] = x;
+        bits = static_cast<unsigned long long>(__double_as_longlong(x));
+        cand = filter && x >= beta;
+      }
+      const unsigned bal = __ballot_sync(kFull, cand);
+      if (bal) {
+        int wbase = 0;
+        if (lane == 0) wbase = atomicAdd(&misc[4], __popc(bal));
+        wbase = __shfl_sync(kFull, wbase, 0);
+        const int slot = wbase + __popc(bal & ((1u << lane) - 1u));
+        if (cand && slot < kEmaCand) {
+          ckey[slot] = bits;
+          cidx[slot] = i;
+        }
+      }
     }
     __syncthreads();
+    const int cnt = misc[4];
+    if (filter && cnt <= kEmaCand) {
+      ranked = true;
+      for (int c = tid; c < cnt; c += blockDim.x) {
+        const unsigned long long kc = ckey[c];
+        const int ic = cidx[c];
+        int rank = 0;
+        for (int j = 0; j < cnt; ++j) {
+          const unsigned long long kj = ckey[j];
+          rank += (kj > kc) | ((kj == kc) & (cidx[j] < ic));
+        }
+        if (rank < peff) atomicOr(&bsel[ic >> 5], 1u << (ic & 31));
+      }
+      __syncthreads();
+    }
   }
   PRR_PHASE(1, u, 1);
 
-  const int peff = min(p.P, nb);
   int* out = p.pred_next + static_cast<size_t>(u) * p.P;
   if (peff <= 0) {
     for (int j = tid; j < p.P; j += blockDim.x) out[j] = -1;
     return;
   }
-  if (peff >= nb) {
+  auto hi = [&](int i) { return static_cast<uint32_t>(static_cast<unsigned long long>(__double_as_longlong(ev[i])) >> 32); };
+  auto lo = [&](int i) { return static_cast<uint32_t>(static_cast<unsigned long long>(__double_as_longlong(ev[i]))); };
+  if (ranked) {
+    // bsel holds the predicted set
+  } else if (peff >= nb) {
     select_bitmap(nb, 0, [&](int) { return 1; }, bsel, beq);
   } else {
     int gt_hi = 0, gt_lo = 0;
-    const uint32_t Thi = radix_kth_largest(
-        nb, peff, [&](int i) { return hi[i]; }, [&](int) { return true; }, hist, misc, &gt_hi);
+    const uint32_t Thi = radix_kth_largest(nb, peff, hi, [&](int) { return true; }, hist, misc, &gt_hi);
     PRR_PHASE(1, u, 2);
     const int need = peff - gt_hi;  // taken from the entries tied on the high word
     // low word among the entries tied on the high word (no pass at all when they agree)
     const uint32_t Tlo = radix_kth_largest(
-        nb, need, [&](int i) { return lo[i]; }, [&](int i) { return hi[i] == Thi; }, hist, misc, &gt_lo);
+        nb, need, lo, [&](int i) { return hi(i) == Thi; }, hist, misc, &gt_lo);
     PRR_PHASE(1, u, 3);
     select_bitmap(
         nb, need - gt_lo,
         [&](int i) {
-          const uint32_t h = hi[i];
+          const uint32_t h = hi(i);
           if (h != Thi) return h > Thi ? 1 : -1;
-          const uint32_t l = lo[i];
+          const uint32_t l = lo(i);
           return l > Tlo ? 1 : (l == Tlo ? 0 : -1);
         },
         bsel, beq);
   }
-  if (warp == 0) warp_emit_bitmap(bsel, nullptr, (nb + 31) / 32, out, p.P);
+  if (warp == 0) warp_emit_bitmap(bsel, nullptr, Wn, out, p.P);
   __syncthreads();
   PRR_PHASE(1, u, 4);
 }

@@ -4,8 +4,8 @@
 // Ranking order everywhere: larger key first, ties broken by the lower index.  The
 // top-k set is therefore {key > T} plus the lowest-index entries with key == T, where
 // T is the k-th largest key (with multiplicity).  T is found MSB-first, 8 bits per
-// pass, from a shared-memory histogram (plain shared atomics: cheaper here than any
-// warp-collective aggregation).  Sets are then held as bitmaps (one ballot per
+// pass, from a shared-memory histogram (shared atomics; the lanes of a warp that agree
+// with its first active lane add in one atomic, which keeps heavy ties cheap).  Sets are then held as bitmaps (one ballot per
 // 32 entries); trimming the ties and writing a set in ascending index order take one
 // warp, popcounts and a shuffle prefix sum.  These routines run once per step on the
 // critical path, so they use few barriers and no CTA-wide scans.  Every thread of the
@@ -71,10 +71,24 @@ __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, 
   for (int shift = 24 - 8 * skip; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += NT) hist[i] = 0u;
     __syncthreads();
-    for (int i = tid; i < n; i += NT) {
-      if (member(i)) {
+    for (int base = 0; base < n; base += NT) {  // warp-uniform trip count
+      const int i = base + tid;
+      unsigned dg = 0u;
+      bool act = false;
+      if (i < n && member(i)) {
         const uint32_t kv = key(i);
-        if ((kv & pmask) == prefix) atomicAdd(&hist[(kv >> shift) & 0xFFu], 1u);
+        act = (kv & pmask) == prefix;
+        dg = (kv >> shift) & 0xFFu;
+      }
+      // Heavily tied keys share a bin: the lanes agreeing with the first active lane
+      // add in one atomic (a per-lane atomic on one address would serialise).
+      const unsigned am = __ballot_sync(kFull, act);
+      if (am) {
+        const int leader = __ffs(am) - 1;
+        const unsigned d0 = __shfl_sync(kFull, dg, leader);
+        const unsigned same = __ballot_sync(kFull, act && dg == d0);
+        if (lane == leader) atomicAdd(&hist[d0], static_cast<unsigned>(__popc(same)));
+        else if (act && dg != d0) atomicAdd(&hist[dg], 1u);
       }
     }
     __syncthreads();

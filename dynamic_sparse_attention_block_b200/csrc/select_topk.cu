@@ -15,8 +15,9 @@
 // Work split: grid (chunk, unit), 256 threads.  Warps 0-3 of each CTA stream 32-block
 // tiles of summaries through private 2-stage shared-memory rings (1-D TMA bulk copies)
 // and score one block per lane; the order-preserving 32-bit keys go to the workspace.
-// The last CTA of a unit to finish (atomic ticket, no waiting) loads the unit's keys,
-// finds the K-th largest by radix selection and emits the selected set in block order.
+// Each warp also writes its 32-block group's largest key and tie mask.  The last CTA of
+// a unit to finish (atomic ticket, no waiting) selects the top K (select_finish) and
+// emits the selected set in block order.
 // In decode-step mode the CTA owning the block of the newly appended token first folds
 // that token into the block's summary (step a1) and writes it back.
 #include "prr_parts.cuh"
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(256, 1) select_topk_kernel(const __grid_consta
     int it = 0;
     for (int r = warp; r < nrounds; r += 4, ++it) {
       const int s = it & 1;
-      if (!mbar_wait(&wbar[s], phase[s], p.status)) {
+      if (!__all_sync(kFull, mbar_wait(&wbar[s], phase[s], p.status))) {  // warp-uniform verdict
         alive = false;
         break;
       }
@@ -107,7 +108,12 @@ __global__ void __launch_bounds__(256, 1) select_topk_kernel(const __grid_consta
       if (own_tail && tail >= first && tail < first + rows)
         fold_tail_row<D>(reinterpret_cast<uint32_t*>(tile + (tail - first) * ROWB), newk, ((n - 1) % p.bs) == 0,
                          reinterpret_cast<uint32_t*>(summ_unit + static_cast<size_t>(tail) * 2 * D), lane);
-      if (lane < rows) keys_out[first + lane] = orderable(score_summary_row<D>(tile + lane * ROWB, coef_lo, coef_hi, lane));
+      uint32_t key = 0u;
+      if (lane < rows) {
+        key = orderable(score_summary_row<D>(tile + lane * ROWB, coef_lo, coef_hi, lane));
+        keys_out[first + lane] = key;
+      }
+      write_group_summary(p, u, first / 32, key, lane < rows);
       __syncwarp();
       if (lane == 0 && r + 8 < nrounds) {
         const uint32_t bytes = min(32, cnt - (r + 8) * 32) * ROWB;

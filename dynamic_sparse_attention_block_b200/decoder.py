@@ -101,8 +101,10 @@ class PRRDecoder:
     def fused_items(self) -> dict:
         """Work-item counts of one fused launch, in queue order."""
         d = self.dims
-        return {"sel": d.units * -(-d.maxnb // 128), "spec": d.units * d.P, "repair": d.units * d.K,
-                "ema": d.units, "combine": d.units * d.G}
+        rep = min(d.K, max(4, -(-1024 // d.units)))
+        chunk = min(128, max(32, -(-(-(-d.units * d.maxnb // 512)) // 32) * 32))
+        return {"sel": d.units * -(-d.maxnb // chunk), "fin": d.units, "ema": d.units,
+                "spec": d.units * d.P, "repair": d.units * rep, "combine": d.units * d.G}
 
     def enable_trace(self, on: bool = True) -> None:
         """Record start/end times of every work item of the fused launches."""

@@ -107,8 +107,10 @@ typedef struct {
   float* lse;
   /* Optional (NULL: off).  prr_decode_step_fused records, for every work item i of the
    * launch, trace[4i..4i+3] = {start ns, end ns, (SM id << 32) | CTA, i} (%globaltimer).
-   * Items, in order: units*ceil(maxnb/128) selection chunks, units*P speculative
-   * slots, units*K repair slots, units predictor updates, units*G merges. */
+   * Items, in order: units*ceil(maxnb/C) selection chunks (C = ceil(units*maxnb/512)
+   * rounded up to a multiple of 32, clamped to [32, 128]), units finishers,
+   * units predictor updates, units*P speculative slots, units*R repair items
+   * (R = min(K, max(4, ceil(1024/units)))), units*G merges. */
   unsigned long long* trace;
 } prr_step_buffers;
 
