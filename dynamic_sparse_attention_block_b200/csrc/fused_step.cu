@@ -9,8 +9,8 @@
 //   4. SPEC    (unit, predicted slot): speculative partial of block Pred_t[slot].  A
 //              speculative item that starts after its unit's selection is published
 //              skips a block that selection dropped (its partial would be discarded).
-//   5. REPAIR  (unit, r < R): partials of the missed blocks in slots r, r + R, ...
-//              (waits for S_t).
+//   5. REPAIR  (unit, r < R): partials of the missed blocks in slots r, r + R, ...;
+//              each slot's block arrives in a descriptor word the finisher publishes.
 //   6. COMBINE (unit, query head): LSE merge of kept + repaired partials (waits for all
 //              of the unit's speculative and repair partials).
 // This is the PRR runtime (abstract; method summary; contributions (1)-(3)) scheduled
@@ -52,13 +52,15 @@ struct FusedCtl {
   unsigned* spec_done;   // [units] finished (or skipped) speculative items
   unsigned* rep_done;    // [units] finished repair items
   unsigned* keepf;       // [units][P] 0 until S_t is known, then 1 | keep << 1
+  unsigned* rdesc;       // [units][K] 0 until S_t is known, then missed block + 1 or kNoRepair
 };
 
 __device__ __forceinline__ FusedCtl ctl_view(const Params& p, int parity) {
   unsigned* b = p.ctl + static_cast<size_t>(parity) * p.ctl_words;
   const int U = p.units;
-  return FusedCtl{b,          b + 1,          b + 2,          b + 3,         b + 16,
-                  b + 16 + U, b + 16 + 2 * U, b + 16 + 3 * U, b + 16 + 4 * U, b + 16 + 5 * U};
+  return FusedCtl{b,          b + 1,          b + 2,          b + 3,          b + 16,
+                  b + 16 + U, b + 16 + 2 * U, b + 16 + 3 * U, b + 16 + 4 * U, b + 16 + 5 * U,
+                  b + 16 + 5 * U + static_cast<size_t>(U) * p.P};
 }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -191,7 +193,8 @@ __device__ void fin_item(const Params& p, const FusedCtl& C, int u, unsigned cha
   if (!wait_geq(C.sel_cnt + u, static_cast<unsigned>(p.fchunks), C, p.status, sh)) return;
   const int n = checked_len(p, u / p.Hkv);
   const int nb = (n + p.bs - 1) / p.bs;
-  const FinishOut f = select_finish(p, u, nb, smem, C.keepf + static_cast<size_t>(u) * p.P);
+  const FinishOut f = select_finish(p, u, nb, smem, C.keepf + static_cast<size_t>(u) * p.P,
+                                    C.rdesc + static_cast<size_t>(u) * p.K);
   __syncthreads();  // every thread's outputs precede the release below
   if (threadIdx.x == 0) {
     C.p_act[u] = static_cast<unsigned>(f.p_active);
@@ -312,17 +315,26 @@ __global__ void __launch_bounds__(128, 3) fused_step_kernel(const __grid_constan
     if (it < n_spec) {  // speculation
       if (tid == 0) next_ticket = atomicAdd(C.work, 1u);
       const int u = it / p.P, j = it % p.P;
+      // the predicted block, the sequence length and the slot's keep flag in one round trip
+      // (the keep flag may change under us: thread 0 reads it and shares its verdict)
+      if (tid == 0) sh[3] = (__ldcg(C.keepf + static_cast<size_t>(u) * p.P + j) == 1u) ? 1 : 0;
+      const int blk = p.pred[static_cast<size_t>(u) * p.P + j];
       const int n = checked_len(p, u / p.Hkv);
       const int nb = (n + BS - 1) / BS;
-      const int blk = p.pred[static_cast<size_t>(u) * p.P + j];
+      __syncthreads();
+      bool dropped = sh[3] != 0;
+      __syncthreads();
       if (blk >= 0 && blk < nb) {
         // speculation has slack; selection is on the critical path.  Gate 1: wait until
         // every selection tile has landed; gate 2: until every unit's S_t is published.
-        if (p.spec_gate == 1) wait_geq(C.sel_loaded, static_cast<unsigned>(n_sel), C, p.status, sh);
-        if (p.spec_gate == 2) wait_geq(C.sel_finished, static_cast<unsigned>(U), C, p.status, sh);
-        if (tid == 0) sh[3] = (__ldcg(C.keepf + static_cast<size_t>(u) * p.P + j) == 1u) ? 1 : 0;  // dropped
-        __syncthreads();
-        const bool skip = sh[3] != 0;
+        if (p.spec_gate != 0) {
+          if (p.spec_gate == 1) wait_geq(C.sel_loaded, static_cast<unsigned>(n_sel), C, p.status, sh);
+          if (p.spec_gate == 2) wait_geq(C.sel_finished, static_cast<unsigned>(U), C, p.status, sh);
+          if (tid == 0) sh[3] = (__ldcg(C.keepf + static_cast<size_t>(u) * p.P + j) == 1u) ? 1 : 0;
+          __syncthreads();
+          dropped = sh[3] != 0;
+        }
+        const bool skip = dropped;
         if (!skip) {
           const size_t row0 = static_cast<size_t>(u) * p.G * p.P + j;
           const PartialDst dst{p.pm + row0, p.pl + row0, p.pO + row0 * D, static_cast<size_t>(p.P),
@@ -340,27 +352,28 @@ __global__ void __launch_bounds__(128, 3) fused_step_kernel(const __grid_constan
     it -= n_spec;
     if (it < n_rep) {  // repair
       if (tid == 0) next_ticket = atomicAdd(C.work, 1u);
-      const int u = it / R, r = it % R;
-      unsigned flag = 0u;
-      if (wait_geq(C.sel_done + u, 1u, C, p.status, sh, &flag)) {
-        const int nm = min(static_cast<int>(flag) - 1, p.K);  // |M_t| came with the flag
-        for (int i = r; i < nm; i += R) {  // missed slots r, r + R, ...
-          const int n = checked_len(p, u / p.Hkv);
-          const int nb = (n + BS - 1) / BS;
-          const int blk = __ldcg(p.missed + static_cast<size_t>(u) * p.K + i);
-          const size_t row0 = static_cast<size_t>(u) * p.G * p.K + i;
-          const PartialDst dst{p.rm + row0, p.rl + row0, p.rO + row0 * D, static_cast<size_t>(p.K),
-                               static_cast<size_t>(p.K) * D};
-          if (blk >= 0 && blk < nb) {
-            if (!block_partial<D, BS>(p, &kmap, &vmap, u, blk, n, dst, smem, bars, ph_attn) && tid == 0)
-              atomicExch(C.abort, 1u);
-            ph_attn ^= 1u;
-          } else {
-            if (tid == 0) report(p.status, kDevBadMissed);
-            write_empty_partial(dst, p.G, D);
-          }
-          count_done(C.rep_done + u);
+      const int u = it / R;
+      const int n = checked_len(p, u / p.Hkv);
+      const int nb = (n + BS - 1) / BS;
+      // slots r, r + R, ...: each slot's descriptor (the missed block + 1, or kNoRepair)
+      // is published by the finisher, so one acquire load hands over the block
+      for (int i = it % R; i < p.K; i += R) {
+        unsigned desc = 0u;
+        if (!wait_geq(C.rdesc + static_cast<size_t>(u) * p.K + i, 1u, C, p.status, sh, &desc)) break;
+        if (desc == kNoRepair) break;
+        const int blk = static_cast<int>(desc) - 1;
+        const size_t row0 = static_cast<size_t>(u) * p.G * p.K + i;
+        const PartialDst dst{p.rm + row0, p.rl + row0, p.rO + row0 * D, static_cast<size_t>(p.K),
+                             static_cast<size_t>(p.K) * D};
+        if (blk >= 0 && blk < nb) {
+          if (!block_partial<D, BS>(p, &kmap, &vmap, u, blk, n, dst, smem, bars, ph_attn) && tid == 0)
+            atomicExch(C.abort, 1u);
+          ph_attn ^= 1u;
+        } else {
+          if (tid == 0) report(p.status, kDevBadMissed);
+          write_empty_partial(dst, p.G, D);
         }
+        count_done(C.rep_done + u);
       }
       __syncthreads();
       if (p.trace && tid == 0) p.trace[4 * static_cast<size_t>(item_id) + 1] = global_ns();

@@ -58,7 +58,7 @@ WsLayout layout_for(const prr_dims* d) {
   L.rO = off;
   off = align256(off + 4 * units * G * d->K * d->d);
   L.ctl = off;
-  off = align256(off + 4 * 2 * (16 + 5 * units + units * static_cast<size_t>(d->P)));
+  off = align256(off + 4 * 2 * (16 + 5 * units + units * static_cast<size_t>(d->P) + units * static_cast<size_t>(d->K)));
   L.total = off;
   return L;
 }
@@ -136,7 +136,7 @@ Params base_params(const prr_dims* d, void* ws) {
     p.rO = reinterpret_cast<float*>(w + L.rO);
     p.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
   }
-  p.ctl_words = 16 + 5 * p.units + p.units * p.P;
+  p.ctl_words = 16 + 5 * p.units + p.units * p.P + p.units * p.K;
   // repair items per unit of the fused step: enough to spread a unit's misses over
   // many CTAs, few enough that empty items (most units miss little) stay cheap
   p.rep_items = std::min(p.K, std::max(4, (1024 + p.units - 1) / p.units));

@@ -29,7 +29,7 @@ struct WsLayout {
   size_t rm;         // float [units*G][K] repair partial max (base-2 logits)
   size_t rl;         // float [units*G][K] repair partial sum
   size_t rO;         // float [units*G][K][d] repair partial numerator
-  size_t ctl;        // uint32 [2][16 + 5*units + units*P] control words of the fused step
+  size_t ctl;        // uint32 [2][16 + 5*units + units*(P + K)] control words of the fused step
   size_t total;
 };
 

@@ -142,7 +142,8 @@ __device__ __forceinline__ void fold_tail_row(uint32_t* row, const uint16_t* new
 // differ in: T keeps a bit when at least K_eff keys are >= the candidate value.  That
 // needs no CTA barrier per step.
 
-constexpr int kBitRegs = 32;  // keys per lane kept in registers by the bit search (nb <= 1024)
+constexpr int kBitRegs = 32;     // keys per lane kept in registers by the bit search (nb <= 1024)
+constexpr int kEagerKeys = 4096;  // up to this many keys are fetched with the group summaries
 
 // Start of the bit search: the bits that the smallest and largest keys share, lower
 // bits zero (every key is >= it).
@@ -170,9 +171,12 @@ __host__ __device__ constexpr size_t finish_scratch_bytes(int maxnb) {
          3 * static_cast<size_t>((maxnb + 31) / 32) * 4;
 }
 
-// keepf (optional, [P]): per predicted slot, 1 | keep << 1 once S_t is known.
+// Optional outputs for the fused step: keepf [P], per predicted slot, 1 | keep << 1;
+// rdesc [K], per missed slot, block + 1 (kNoRepair past the last missed block).
+constexpr unsigned kNoRepair = 0xFFFFFFFFu;
+
 __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsigned char* scratch,
-                                          unsigned* keepf = nullptr) {
+                                          unsigned* keepf = nullptr, unsigned* rdesc = nullptr) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, NT = blockDim.x;
   const int W = (p.maxnb + 31) / 32;
   int* spred = reinterpret_cast<int*>(scratch + 256 * 4);  // [128]
@@ -193,7 +197,8 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
   if (use_gs) {
     const uint2* src = p.gsum + static_cast<size_t>(u) * W;
     for (int g = tid; g < Wn; g += NT) gs[g] = __ldcg(src + g);
-  } else if (!take_all) {
+  }
+  if (!take_all && nb <= kEagerKeys) {  // with the summaries: no second round trip if no tie
     load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb);
     have_keys = true;
   }
@@ -241,7 +246,7 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
       T = gmax;
       tie_masks = use_gs;
     } else {
-      if (!have_keys) {
+      if (!have_keys && !take_all) {
         load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb);
         have_keys = true;
         __syncthreads();
@@ -266,12 +271,27 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
           hi = __reduce_max_sync(kFull, hi);
           t = bit_search_start(lo, hi);
           if (lo != hi) {
-            for (int bit = 31 - __clz(lo ^ hi); bit >= 0; --bit) {
-              const uint32_t c = t | (1u << bit);
-              int cnt = 0;
+            int bit = 31 - __clz(lo ^ hi);
+            // two bits per round: three candidate counts, reduced independently
+            for (; bit >= 1; bit -= 2) {
+              const uint32_t c1 = t | (1u << (bit - 1)), c2 = t | (2u << (bit - 1)), c3 = t | (3u << (bit - 1));
+              int n1 = 0, n2 = 0, n3 = 0;
 #pragma unroll
-              for (int q = 0; q < kBitRegs; ++q) cnt += kr[q] >= c ? 1 : 0;
-              if (__reduce_add_sync(kFull, cnt) >= static_cast<unsigned>(keff)) t = c;
+              for (int q = 0; q < kBitRegs; ++q) {
+                n1 += kr[q] >= c1 ? 1 : 0;
+                n2 += kr[q] >= c2 ? 1 : 0;
+                n3 += kr[q] >= c3 ? 1 : 0;
+              }
+              const int s1 = __reduce_add_sync(kFull, n1), s2 = __reduce_add_sync(kFull, n2);
+              const int s3 = __reduce_add_sync(kFull, n3);
+              t = s3 >= keff ? c3 : (s2 >= keff ? c2 : (s1 >= keff ? c1 : t));
+            }
+            if (bit == 0) {
+              const uint32_t c = t | 1u;
+              int n1 = 0;
+#pragma unroll
+              for (int q = 0; q < kBitRegs; ++q) n1 += kr[q] >= c ? 1 : 0;
+              if (__reduce_add_sync(kFull, n1) >= keff) t = c;
             }
           }
           int g = 0;
@@ -360,7 +380,19 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
   if (warp == 0) {
     warp_emit_bitmap(bm_sel, nullptr, Wn, p.sel + static_cast<size_t>(u) * p.K, p.K);
   } else if (warp == 1) {
-    nm = warp_emit_bitmap(bm_sel, bm_pred, Wn, p.missed + static_cast<size_t>(u) * p.K, p.K);
+    // missed list; each missed block is handed to its repair slot and, since the repair
+    // reads it next, started toward L2
+    nm = warp_emit_bitmap(bm_sel, bm_pred, Wn, p.missed + static_cast<size_t>(u) * p.K, p.K, [&](int pos, int b) {
+      if (rdesc) rdesc[pos] = static_cast<unsigned>(b) + 1u;
+      if (p.kc && p.vc) {
+        const int rows = min(p.bs, p.cap - b * p.bs);
+        const size_t off = (static_cast<size_t>(u) * p.cap + static_cast<size_t>(b) * p.bs) * p.d;
+        prefetch_l2(p.kc + off, static_cast<uint32_t>(rows) * p.d * 2);
+        prefetch_l2(p.vc + off, static_cast<uint32_t>(rows) * p.d * 2);
+      }
+    });
+    if (rdesc)
+      for (int e = nm + lane; e < p.K; e += 32) rdesc[e] = kNoRepair;
     if ((tid & 31) == 0) {
       p.n_missed[u] = nm;
       misc[2] = nm;

@@ -181,9 +181,11 @@ __device__ void select_bitmap(int n, int take_equal, CmpFn cmp, unsigned* bm, un
 }
 
 // One warp.  Write the set bits of bm[0..W) (optionally masked by ~exclude) as
-// ascending indices to out[0..), then -1 up to `cap`.  Returns the count.
-__device__ __forceinline__ int warp_emit_bitmap(const unsigned* bm, const unsigned* exclude, int W, int* out,
-                                                int cap) {
+// ascending indices to out[0..), then -1 up to `cap`; on_emit(pos, index) is called
+// for every index written.  Returns the count.
+template <typename EmitFn>
+__device__ __forceinline__ int warp_emit_bitmap(const unsigned* bm, const unsigned* exclude, int W, int* out, int cap,
+                                                EmitFn on_emit) {
   const int lane = threadIdx.x & 31;
   int base = 0;
   for (int w0 = 0; w0 < W; w0 += 32) {
@@ -194,7 +196,10 @@ __device__ __forceinline__ int warp_emit_bitmap(const unsigned* bm, const unsign
     int pos = base + inc - c;
     while (b) {
       const int bit = __ffs(b) - 1;
-      if (pos < cap) out[pos] = wd * 32 + bit;
+      if (pos < cap) {
+        out[pos] = wd * 32 + bit;
+        on_emit(pos, wd * 32 + bit);
+      }
       ++pos;
       b &= b - 1u;
     }
@@ -202,6 +207,11 @@ __device__ __forceinline__ int warp_emit_bitmap(const unsigned* bm, const unsign
   }
   for (int e = base + lane; e < cap; e += 32) out[e] = -1;
   return base;
+}
+
+__device__ __forceinline__ int warp_emit_bitmap(const unsigned* bm, const unsigned* exclude, int W, int* out,
+                                                int cap) {
+  return warp_emit_bitmap(bm, exclude, W, out, cap, [](int, int) {});
 }
 
 }  // namespace prr
