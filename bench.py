@@ -259,7 +259,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    w = W.workload(args.workload)
+    w = base_workload(args)
     threads = os.cpu_count() or 1
     value, sps, nsteps, units, used = oracle_run(w, args.warmup, args.steps, args.ref_budget_s, threads)
     line = {
@@ -276,6 +276,12 @@ def run_reference(args):
         line["note"] = f"timed {nsteps} of {args.steps} requested steps (time budget {args.ref_budget_s}s)"
     print(json.dumps(line), flush=True)
     return 0
+
+
+def base_workload(args) -> W.Workload:
+    w = W.workload(args.workload)
+    batch = getattr(args, "batch", 0)
+    return w.with_(B=batch) if batch > 0 else w
 
 
 def workload_config(w: W.Workload, args) -> dict:
@@ -298,14 +304,14 @@ def run_gpu(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    w = rank_workload(W.workload(args.workload), rank)
+    w = rank_workload(base_workload(args), rank)
     hbm_peak, peak_kind = measured_peaks()
 
     # CPU baseline first (rank 0, N = 1 only), before any GPU work
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
-        value, sps, nsteps, units, used = oracle_run(W.workload(args.workload), 2, args.cpu_max_steps,
+        value, sps, nsteps, units, used = oracle_run(base_workload(args), 2, args.cpu_max_steps,
                                                      args.cpu_budget_s, threads)
         cpu = {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                "sample": f"{nsteps} oracle decode steps of {w.name} after 2 warm-up steps "
@@ -586,6 +592,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("prr", "reference"), default="prr")
     ap.add_argument("--workload", default="llama8b_32k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (reduced cases for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-streams", action="store_true", help="skip the two-stream comparison run")
