@@ -203,33 +203,6 @@ __device__ void fin_item(const Params& p, const FusedCtl& C, int u, unsigned cha
   }
 }
 
-// ---------------------------------------------------------------- L2 prefetch
-// Items are handed out roughly round-robin, so item it + gridDim.x is about one round
-// ahead.  Asking L2 for its data now keeps HBM busy while CTAs compute; every byte is
-// still read once from HBM (the item later finds it in L2).  Only SEL and SPEC items
-// have addresses known before the launch ends selection.
-template <int D, int BS>
-__device__ __forceinline__ void prefetch_item(const Params& p, int ahead, int n_sel, int spec0, int n_spec) {
-  if (ahead < n_sel) {
-    const int u = ahead / p.fchunks, c0 = (ahead % p.fchunks) * p.fchunk_blocks;
-    const int rows = min(p.fchunk_blocks, p.maxnb - c0);
-    if (rows > 0)
-      prefetch_l2(p.summ + (static_cast<size_t>(u) * p.maxnb + c0) * 2 * D, static_cast<uint32_t>(rows) * 4 * D);
-  } else if (ahead >= spec0 && ahead < spec0 + n_spec) {
-    const int s = ahead - spec0, u = s / p.P, j = s % p.P;
-    const int blk = __ldg(p.pred + static_cast<size_t>(u) * p.P + j);  // read-only in this launch
-    if (blk >= 0 && blk < p.maxnb) {
-      const int t0 = blk * BS;
-      const int rows = min(BS, p.cap - t0);
-      if (rows > 0) {
-        const size_t off = (static_cast<size_t>(u) * p.cap + t0) * D;
-        prefetch_l2(p.kc + off, static_cast<uint32_t>(rows) * D * 2);
-        prefetch_l2(p.vc + off, static_cast<uint32_t>(rows) * D * 2);
-      }
-    }
-  }
-}
-
 // ---------------------------------------------------------------- fused kernel
 template <int D, int BS>
 __global__ void __launch_bounds__(128, 3) fused_step_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -288,7 +261,6 @@ __global__ void __launch_bounds__(128, 3) fused_step_kernel(const __grid_constan
       p.trace[4 * static_cast<size_t>(it) + 3] = static_cast<unsigned long long>(it);
     }
     const int item_id = it;
-    if (tid == 32) prefetch_item<D, BS>(p, it + static_cast<int>(gridDim.x), n_sel, n_sel + n_fin + n_ema, n_spec);
 
     if (it < n_sel) {
       if (tid == 0) next_ticket = atomicAdd(C.work, 1u);

@@ -148,6 +148,7 @@ Params base_params(const prr_dims* d, void* ws) {
     }
     p.spec_gate = gate;
   }
+
   return p;
 }
 

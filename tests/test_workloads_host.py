@@ -1,0 +1,67 @@
+"""Host-side logic on CPU: the seeded input generators and the bench's byte accounting.
+
+The generators feed both the oracle and the CUDA path, so their contract (exact bf16
+rounding, the forced-overlap construction, determinism) is checked on its own here.
+"""
+import numpy as np
+import pytest
+
+import bench
+import workloads as W
+
+
+def test_bf16_round_to_nearest_even():
+    x = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.5, 0.0], np.float32)
+    bits = W.f32_to_bf16_bits(x)
+    # 1 + 2^-8 is a tie between 1 and 1 + 2^-7: even mantissa (1.0) wins; 1 + 3*2^-8 rounds up
+    assert bits.tolist() == [0x3F80, 0x3F80, 0x3F82, 0xC020, 0x0000]
+    assert np.array_equal(W.bf16_bits_to_f32(bits), np.array([1.0, 1.0, 1.0 + 2.0 ** -6, -2.5, 0.0], np.float32))
+
+
+def test_grid_values_and_determinism():
+    w = W.workload("tiny")
+    q1, q2 = W.queries(w, 4), W.queries(w, 4)
+    assert np.array_equal(q1, q2)
+    vals = W.bf16_bits_to_f32(q1).ravel() * 8
+    assert np.all(vals == np.round(vals)) and vals.min() >= -8 and vals.max() <= 8
+    k, v = W.kv_prefix(w, 0, 0, 256)
+    kv = W.bf16_bits_to_f32(k) * 8
+    assert np.all(kv == np.round(kv))
+    assert np.abs(W.bf16_bits_to_f32(v)).max() < 8  # N(0,1) values, not grid
+
+
+def test_query_walk_keeps_most_channels():
+    w = W.workload("llama8b_32k")
+    q = W.queries(w, 8)
+    same = np.mean(q[1:] == q[:-1])
+    # kept with probability 0.9, or redrawn to the same grid value (1/17)
+    assert 0.85 < same < 0.97
+
+
+@pytest.mark.parametrize("overlap,kept", [(1.0, 64), (0.97, 62), (0.9, 58), (0.75, 48), (0.5, 32), (0.0, 0)])
+def test_forced_prediction_overlap(overlap, kept):
+    w = W.workload("repair_sweep_64k")
+    rng = np.random.default_rng(3)
+    nb = 1025
+    sel = np.sort(rng.choice(nb, size=64, replace=False))
+    assert W.forced_kept_count(overlap, 64) == kept
+    fp = W.forced_prediction(w, sel, nb, overlap, 1, 5, 2, 3)
+    assert len(fp) == 64 and np.all(np.diff(fp) > 0) and fp.min() >= 0 and fp.max() < nb
+    assert len(np.intersect1d(fp, sel)) == kept
+    assert np.array_equal(fp, W.forced_prediction(w, sel, nb, overlap, 1, 5, 2, 3))
+
+
+@pytest.mark.parametrize("name,mb", [("llama8b_32k", 18.88), ("batched_128k", 335.6), ("long_512k", 201.3)])
+def test_algorithmic_bytes(name, mb):
+    # summaries of every block (2d bf16 each) + K and V of the K_eff selected blocks
+    w = W.workload(name)
+    b = bench.algorithmic_bytes(w, w.N0 + 1)
+    assert b["total"] == b["summaries"] + b["kv"]
+    assert abs(b["total"] / 1e6 - mb) < 0.05 * mb
+
+
+def test_batch_override_for_reduced_captures():
+    class A:
+        workload, batch = "batched_128k", 6
+    w = bench.base_workload(A())
+    assert w.B == 6 and w.N0 == W.workload("batched_128k").N0
