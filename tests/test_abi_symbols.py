@@ -64,3 +64,19 @@ def test_argument_checks_return_before_any_launch(lib):
     st = lib.prr_select_topk_static(ctypes.byref(big), fake, fake, fake, fake, fake, fake, fake, fake,
                                     null, null)
     assert st == 3
+
+
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++17")])
+def test_header_compiles_standalone(tmp_path, lang, std):
+    """include/prr.h is a plain C header: it compiles on its own as C99 and as C++."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = tmp_path / ("t.c" if lang == "c" else "t.cpp")
+    src.write_text('#include "prr.h"\nint main(void) { prr_dims d = {0}; (void)d; return PRR_OK; }\n')
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-Werror", f"-std={std}", "-I", os.path.join(ROOT, "include"),
+                        "-I", cuda_inc, str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
