@@ -266,7 +266,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": nsteps, "warmup": args.warmup, "ms_per_step": sps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, args),
+        "config": dict(workload_config(w, args), l2="not applicable (host CPU)"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                          "sample": f"{nsteps} full oracle decode steps ({units} (sequence, KV head) "
                                    f"units each) of {w.name}, OpenMP over units"},
@@ -507,36 +507,35 @@ def run_gpu(args):
     # ---------------- end to end: host buffers through the public API
     e2e = None
     if e2e_steps:
-        q_h = torch.from_numpy(qs.view(np.int16)).view(torch.bfloat16).pin_memory()
-        kn_h = torch.from_numpy(kn.view(np.int16)).view(torch.bfloat16).pin_memory()
-        vn_h = torch.from_numpy(vn.view(np.int16)).view(torch.bfloat16).pin_memory()
-        out_h = torch.empty(dec.out.shape, dtype=torch.float32).pin_memory()
-        lse_h = torch.empty(dec.lse.shape, dtype=torch.float32).pin_memory()
-        k_stage = torch.empty_like(kn_d[0])
-        v_stage = torch.empty_like(vn_d[0])
+        # the step's inputs as the decoder lays them out: [q | k_new | v_new], one pinned
+        # host row per step; outputs [out | lse] come back in one copy
+        nq, nkv = dec.q.numel(), dec.k_new.numel()
+        in_h = torch.empty((total, nq + 2 * nkv), dtype=torch.bfloat16).pin_memory()
+        in_h[:, :nq] = torch.from_numpy(qs.reshape(total, -1).view(np.int16)).view(torch.bfloat16)
+        in_h[:, nq:nq + nkv] = torch.from_numpy(kn.reshape(total, -1).view(np.int16)).view(torch.bfloat16)
+        in_h[:, nq + nkv:] = torch.from_numpy(vn.reshape(total, -1).view(np.int16)).view(torch.bfloat16)
+        out_h = torch.empty(dec.io_out.shape, dtype=torch.float32).pin_memory()
         e_tokens = 0
         es = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
         ee = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
         for i in range(e2e_steps):
             flush.zero_()
             es[i].record(main)
-            dec.q.copy_(q_h[t], non_blocking=True)
-            k_stage.copy_(kn_h[t], non_blocking=True)
-            v_stage.copy_(vn_h[t], non_blocking=True)
-            dec.append(k_stage, v_stage, stream=main)
+            dec.io_in.copy_(in_h[t], non_blocking=True)
+            dec.append(dec.k_new, dec.v_new, stream=main)
             replay("fused")
-            out_h.copy_(dec.out, non_blocking=True)
-            lse_h.copy_(dec.lse, non_blocking=True)
+            out_h.copy_(dec.io_out, non_blocking=True)
             ee[i].record(main)
             main.synchronize()
             e_tokens += w.B * (w.N0 + t + 1)
             t += 1
         e_ms = [a.elapsed_time(b) for a, b in zip(es, ee)]
-        h2d = q_h[0].numel() * 2 + kn_h[0].numel() * 2 * 2
-        d2h = out_h.numel() * 4 + lse_h.numel() * 4
+        h2d = in_h[0].numel() * 2
+        d2h = out_h.numel() * 4
         e2e = {"value": e_tokens / (sum(e_ms) / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": statistics.mean(e_ms),
-               "path": "append + fused step graph + D2H of out/lse, pinned host buffers"}
+               "path": "one H2D of [q | k_new | v_new], append, fused step graph, one D2H of "
+                       "[out | lse]; pinned host buffers"}
         if not np.all(np.isfinite(out_h.numpy())):
             status = status or -1
 

@@ -46,9 +46,16 @@ class PRRDecoder:
         self.part_m = torch.zeros((B, Hq, max(P, 1)), dtype=torch.float32, device=dev)
         self.part_l = torch.zeros((B, Hq, max(P, 1)), dtype=torch.float32, device=dev)
         self.part_O = torch.zeros((B, Hq, max(P, 1), d), dtype=torch.float32, device=dev)
-        self.out = torch.zeros((B, Hq, d), dtype=torch.float32, device=dev)
-        self.lse = torch.zeros((B, Hq), dtype=torch.float32, device=dev)
-        self.q = torch.zeros((B, Hq, d), dtype=torch.bfloat16, device=dev)
+        # Per-step I/O in two contiguous buffers, so that a caller moves each direction
+        # with one copy: io_in = [q | k_new | v_new] (bf16), io_out = [out | lse] (fp32).
+        nq, nkv = B * Hq * d, B * Hkv * d
+        self.io_in = torch.zeros((nq + 2 * nkv,), dtype=torch.bfloat16, device=dev)
+        self.q = self.io_in[:nq].view(B, Hq, d)
+        self.k_new = self.io_in[nq:nq + nkv].view(B, Hkv, d)
+        self.v_new = self.io_in[nq + nkv:].view(B, Hkv, d)
+        self.io_out = torch.zeros((B * Hq * (d + 1),), dtype=torch.float32, device=dev)
+        self.out = self.io_out[:B * Hq * d].view(B, Hq, d)
+        self.lse = self.io_out[B * Hq * d:].view(B, Hq)
         nbytes = _abi.prr_workspace_bytes(dims)
         if nbytes == 0:
             raise ValueError(f"unsupported dims {dims}")
