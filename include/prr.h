@@ -142,7 +142,8 @@ const char* prr_status_string(prr_status s);
 
 /* Bytes of workspace the calls below need for these dims (0 if the dims are
  * unsupported).  The workspace holds the status word, the selection tickets, one
- * 32-bit score key per block and the repair partials. */
+ * 32-bit score key per block, one (max key, tie mask) summary per 32-block group, the
+ * repair partials and the fused step's control words (two copies, one per parity). */
 size_t prr_workspace_bytes(const prr_dims* dims);
 
 /* Zero-fill a workspace (required once before first use, and after a device error).
