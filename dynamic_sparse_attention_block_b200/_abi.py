@@ -47,7 +47,7 @@ SYMBOLS = (
     "prr_version", "prr_status_string", "prr_workspace_bytes", "prr_workspace_init",
     "prr_get_device_status", "prr_append_kv", "prr_update_summaries", "prr_select_topk",
     "prr_ema_predict", "prr_speculate", "prr_repair_merge", "prr_decode_step",
-    "prr_decode_step_fused", "prr_select_topk_static",
+    "prr_decode_step_fused", "prr_budget_fit", "prr_budget_choose", "prr_select_topk_static",
 )
 
 # mirrors PRR_SELECT_STATIC_MAX_BLOCKS / PRR_SELECT_STATIC_SCRATCH_BYTES in include/prr.h
@@ -101,6 +101,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
                                   ctypes.POINTER(PrrStepEvents)]
     L.prr_decode_step_fused.argtypes = [dims, ctypes.POINTER(PrrStepBuffers), vp, sz, _i32, vp]
     L.prr_select_topk_static.argtypes = [dims, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.prr_budget_fit.argtypes = [vp, vp, _i32, _i32, vp]
+    L.prr_budget_choose.argtypes = [vp, vp, vp, _i32, _i32, _i32, ctypes.POINTER(_i32)]
     for name in SYMBOLS:
         if name not in ("prr_version", "prr_status_string", "prr_workspace_bytes"):
             getattr(L, name).restype = ctypes.c_int
@@ -224,6 +226,33 @@ def prr_select_topk_static(dims, q, summ, seq_lens, pred, sel, missed, n_missed,
                                          _ptr(pred), _ptr(sel), _ptr(missed), _ptr(n_missed),
                                          _ptr(keep), _ptr(status), _stream(stream)),
            "prr_select_topk_static")
+
+
+def prr_budget_fit(context_tokens, us, degree: int):
+    """Least-squares polynomial (lowest order first) of us against context length."""
+    import numpy as np
+    x = np.ascontiguousarray(context_tokens, dtype=np.float64)
+    y = np.ascontiguousarray(us, dtype=np.float64)
+    if x.shape != y.shape or x.ndim != 1:
+        raise ValueError("context_tokens and us must be 1-D and of one length")
+    coef = np.zeros(degree + 1 if degree >= 0 else 1, dtype=np.float64)
+    _check(load().prr_budget_fit(x.ctypes.data, y.ctypes.data, len(x), int(degree), coef.ctypes.data),
+           "prr_budget_fit")
+    return coef
+
+
+def prr_budget_choose(sel_coef, spec_coef, p_grid, context_tokens: int) -> int:
+    """Largest profiled budget whose predicted speculation time fits in selection's."""
+    import numpy as np
+    sc = np.ascontiguousarray(sel_coef, dtype=np.float64)
+    pc = np.ascontiguousarray(spec_coef, dtype=np.float64)
+    pg = np.ascontiguousarray(p_grid, dtype=np.int32)
+    if pc.ndim != 2 or pc.shape != (len(pg), len(sc)):
+        raise ValueError("spec_coef must be [len(p_grid)][degree+1]")
+    out = _i32(0)
+    _check(load().prr_budget_choose(sc.ctypes.data, pc.ctypes.data, pg.ctypes.data, len(pg), len(sc) - 1,
+                                    int(context_tokens), ctypes.byref(out)), "prr_budget_choose")
+    return int(out.value)
 
 
 def prr_ema_predict(dims, ema, sel, seq_lens, pred_next, ws, stream=None) -> None:

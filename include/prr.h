@@ -245,6 +245,26 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* buf, vo
 prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* buf, void* ws,
                                  size_t ws_bytes, int32_t step_parity, cudaStream_t stream);
 
+/* Profiling-guided speculation budget (PRR abstract: the speculation budget comes from
+ * profiling and keeps speculative work off the critical path; limitations: overheads
+ * at context lengths between the profiled points come from polynomial regressions).
+ * Host functions: they touch no device memory and need no GPU.
+ *
+ * prr_budget_fit: least-squares polynomial of degree `degree` (0..3) through the n
+ * points (context_tokens[i], us[i]), in x = context_tokens / 65536; coef[0..degree]
+ * receives the coefficients, lowest order first.  PRR_ERR_SHAPE if n <= degree or the
+ * degree is outside 0..3; PRR_ERR_INVALID_ARG for a null pointer or a singular system
+ * (fewer distinct contexts than coefficients). */
+prr_status prr_budget_fit(const double* context_tokens, const double* us, int32_t n, int32_t degree,
+                          double* coef);
+
+/* prr_budget_choose: the speculation budget for a context of context_tokens: the largest
+ * p_grid[j] whose predicted speculation time (polynomial spec_coef[j], [np][degree+1])
+ * does not exceed the predicted selection time (polynomial sel_coef, [degree+1]), or 0
+ * if none does.  p_grid must be strictly ascending.  *p_out receives the budget. */
+prr_status prr_budget_choose(const double* sel_coef, const double* spec_coef, const int32_t* p_grid,
+                             int32_t np, int32_t degree, int32_t context_tokens, int32_t* p_out);
+
 /* Largest B*Hkv*ceil(cap_tokens/bs) that prr_select_topk_static accepts, and the bytes
  * of device memory its fixed scratch array occupies on every GPU that loads the
  * library (status word + 65536 chunk tickets + one 32-bit key per block). */
