@@ -306,6 +306,22 @@ def test_decode_repair_sweep_small(mode):
         _assert_ok(run_parity(w, steps=3, forced=(ov, level), mode=mode))
 
 
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("d,bs,G,K,P", [
+    (64, 64, 8, 128, 128),    # largest K and P (below nb), 8:1 GQA, small head dim
+    (64, 128, 8, 128, 128),   # the same with large blocks: K and P above nb (take all)
+    (128, 64, 1, 1, 1),       # smallest K and P, no grouping
+    (64, 64, 3, 33, 17),      # odd group size, K and P not multiples of 32
+    (128, 128, 5, 100, 128),  # P > K
+])
+def test_decode_shape_limits(mode, d, bs, G, K, P):
+    """Shapes at the limits the ABI accepts (d in {64, 128}, bs in {64, 128}, G <= 8,
+    K and P up to 128), several steps, all units, both step implementations."""
+    w = W.workload("tiny").with_(name="limits", B=2, Hq=2 * G, Hkv=2, d=d, N0=9000 + 37, bs=bs, K=K,
+                                 P=P, steps=4, walk_p=0.8)
+    _assert_ok(run_parity(w, steps=4, mode=mode))
+
+
 @pytest.mark.parametrize("name,steps,units", [
     ("batched_128k", 3, [(0, 0), (7, 3), (15, 7)]),
     ("long_512k", 3, [(0, 0), (2, 5), (3, 7)]),
