@@ -64,6 +64,9 @@ class Oracle:
         L.oracle_build_summaries.argtypes = [_u16p, _int, _int, _int, _f64p, _f64p]
         L.oracle_block_scores.argtypes = [_f64p, _int, _int, _f64p, _f64p, _int, _f64p]
         L.oracle_top_ranked.argtypes = [_f64p, _int, _int, _i32p]
+        L.oracle_block_scores_max.argtypes = [_f64p, _int, _int, _f64p, _f64p, _int, _f64p]
+        L.oracle_top_ranked_forced.argtypes = [_f64p, _int, _int, _int, _int, _i32p]
+        L.oracle_top_ranked_forced.restype = _int
         L.oracle_top_ranked.restype = _int
         L.oracle_ema_update.argtypes = [_f64p, _int, _i32p, _int, _dbl]
         L.oracle_attend_blocks.argtypes = [_f64p, _u16p, _u16p, _int, _int, _int, _i32p, _int,
@@ -114,6 +117,27 @@ class Oracle:
         out = np.full(max(K, 1), -1, dtype=np.int32)
         cnt = self.L.oracle_top_ranked(values, len(values), K, out)
         return out[:cnt].copy()
+
+    def block_scores_max(self, q, smin, smax) -> np.ndarray:
+        """Selector variant: the largest per-head bound of the group (instead of the sum)."""
+        q = _c(q, np.float64)
+        G, d = q.shape
+        nb = smin.shape[0]
+        out = np.zeros(nb, np.float64)
+        self.L.oracle_block_scores_max(q, G, d, _c(smin, np.float64), _c(smax, np.float64), nb, out)
+        return out
+
+    def top_ranked_forced(self, values, K, n_sink, n_local) -> np.ndarray:
+        """Selector variant: first n_sink and last n_local blocks forced, best of the rest."""
+        v = _c(values, np.float64)
+        out = np.zeros(max(min(K, len(v)), 1), np.int32)
+        cnt = self.L.oracle_top_ranked_forced(v, len(v), K, n_sink, n_local, out)
+        return out[:cnt]
+
+    def select_per_head(self, q, smin, smax, K):
+        """Selector variant: every query head selects with its own bound (no sharing)."""
+        q = _c(q, np.float64)
+        return [self.top_ranked(self.block_scores(q[h:h + 1], smin, smax), K) for h in range(q.shape[0])]
 
     def ema_update(self, e, nb, sel, alpha) -> np.ndarray:
         e = _c(e, np.float64).copy()

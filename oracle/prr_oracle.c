@@ -151,6 +151,68 @@ int oracle_top_ranked(const double *v, int nb, int K, int32_t *out)
     return keff;
 }
 
+/* ------------------------------------------------------------------ selector variants
+ *
+ * The abstract measures PRR across "representative DSA methods", whose selectors differ
+ * from the one above.  Two of them, as plain definitions (the pages print no formula;
+ * readings taken):
+ *  - group score as the LARGEST of the per-head bounds instead of their sum;
+ *  - forced blocks: the first n_sink blocks (attention sinks) and the last n_local
+ *    blocks (the local window) are always in S; the rest of the min(K, nb) budget
+ *    goes to the best remaining blocks under (score desc, index asc).  When the forced
+ *    blocks alone exceed the budget, sinks are taken first, lowest index first, then
+ *    local blocks from the newest backwards, until the budget is full.
+ * Per-query-head selection needs nothing new: each head's own bound (G = 1) and top-K. */
+
+/* s_b = max over the G query heads of sum_c max(q_hc*min_bc, q_hc*max_bc). */
+void oracle_block_scores_max(const double *q, int G, int d, const double *smin,
+                             const double *smax, int nb, double *s)
+{
+    for (int b = 0; b < nb; ++b) {
+        double best = 0.0;
+        for (int h = 0; h < G; ++h) {
+            double u = 0.0;
+            for (int c = 0; c < d; ++c) {
+                double lo = q[h * d + c] * smin[(size_t)b * d + c];
+                double hi = q[h * d + c] * smax[(size_t)b * d + c];
+                u += (lo > hi) ? lo : hi;
+            }
+            if (h == 0 || u > best) best = u;
+        }
+        s[b] = best;
+    }
+}
+
+/* Forced sink and local blocks plus the best of the rest; ascending output; returns
+ * the count (min(K, nb)). */
+int oracle_top_ranked_forced(const double *v, int nb, int K, int n_sink, int n_local,
+                             int32_t *out)
+{
+    int keff = K < nb ? K : nb;
+    if (keff <= 0) return 0;
+    unsigned char *taken = (unsigned char *)calloc((size_t)nb, 1);
+    int cnt = 0;
+    for (int b = 0; b < n_sink && b < nb && cnt < keff; ++b)
+        if (!taken[b]) { taken[b] = 1; out[cnt++] = b; }
+    for (int i = 0; i < n_local && cnt < keff; ++i) {
+        int b = nb - 1 - i;
+        if (b < 0) break;
+        if (!taken[b]) { taken[b] = 1; out[cnt++] = b; }
+    }
+    while (cnt < keff) {
+        int best = -1;
+        for (int b = 0; b < nb; ++b) {
+            if (taken[b]) continue;
+            if (best < 0 || ranks_before(v[b], b, v[best], best)) best = b;
+        }
+        taken[best] = 1;
+        out[cnt++] = best;
+    }
+    free(taken);
+    sort_ascending(out, keff);
+    return keff;
+}
+
 /* ------------------------------------------------------------------ 5. EMA */
 
 /* e_b <- alpha*e_b + beta*[b in S] for every b < nb, beta = 1 - alpha. */
