@@ -213,6 +213,17 @@ def reduce_over_ranks(tokens: float, seconds: float, e2e_value, world: int, devi
 
 # ----------------------------------------------------------------------------- CPU oracle timing
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for ln in fh:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_run(w: W.Workload, warmup: int, steps: int, budget_s: float, nthreads: int):
     """Time the fp64 oracle's decode step on the host.  Returns (tokens/s, seconds per
     step, steps timed, units per step, threads).  Each step runs every (sequence, KV
@@ -269,7 +280,8 @@ def run_reference(args):
         "config": dict(workload_config(w, args), l2="not applicable (host CPU)"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                          "sample": f"{nsteps} full oracle decode steps ({units} (sequence, KV head) "
-                                   f"units each) of {w.name}, OpenMP over units"},
+                                   f"units each) of {w.name}, OpenMP over units",
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     if nsteps < args.steps:
@@ -315,7 +327,11 @@ def run_gpu(args):
                                                      args.cpu_budget_s, threads)
         cpu = {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                "sample": f"{nsteps} oracle decode steps of {w.name} after 2 warm-up steps "
-                         f"({units} units per step, ~{args.cpu_budget_s:.0f} s budget)"}
+                         f"({units} units per step, ~{args.cpu_budget_s:.0f} s budget)",
+               "cpu_model": cpu_model()}
+        v1, _, n1, _, _ = oracle_run(base_workload(args), 1, args.cpu_max_steps, args.cpu_budget_s / 3, 1)
+        cpu["single_thread"] = {"value": v1, "unit": UNIT, "cores": 1,
+                                "sample": f"{n1} oracle decode steps, one thread"}
 
     e2e_steps = 0 if args.no_e2e else args.steps
     cmp_steps = 0 if args.no_streams else min(args.steps, 100)
