@@ -118,6 +118,12 @@ class PRRDecoder:
         self.trace = torch.zeros((sum(self.fused_items().values()), 4), dtype=torch.int64,
                                  device=self.device) if on else None
 
+    def trace_summary(self) -> dict:
+        """Timeline of the last traced fused launch, per item kind (see summarize_trace)."""
+        if self.trace is None:
+            raise RuntimeError("tracing is off: call enable_trace() before the step")
+        return summarize_trace(self.trace.cpu().numpy(), self.fused_items())
+
     # ------------------------------------------------------------------ setup
     def prefill(self, k: torch.Tensor, v: torch.Tensor, n0: int) -> None:
         """Copy an initial context of n0 tokens ([B][Hkv][n0][d] bf16) into the cache,
@@ -174,3 +180,32 @@ class PRRDecoder:
 
     def device_status(self) -> int:
         return _abi.prr_get_device_status(self.ws)
+
+
+def summarize_trace(trace, items: dict) -> dict:
+    """Per item kind of one fused launch: how many items ran, when the first and last
+    started and the last ended (microseconds after the earliest start), and the p50 /
+    mean / max item duration.  `trace` is the [items][4] record of prr_step_buffers
+    (start ns, end ns, SM << 32 | CTA, item), `items` the kind counts in queue order."""
+    import numpy as np
+    tr = np.asarray(trace, dtype=np.int64)
+    ran = tr[:, 0] > 0
+    if not ran.any():
+        return {}
+    t0 = tr[ran, 0].min()
+    out, off = {}, 0
+    for kind, cnt in items.items():
+        seg = tr[off:off + cnt]
+        off += cnt
+        seg = seg[seg[:, 0] > 0]
+        if len(seg) == 0:
+            out[kind] = {"n": 0}
+            continue
+        st = (seg[:, 0] - t0) / 1e3
+        en = (seg[:, 1] - t0) / 1e3
+        dur = en - st
+        out[kind] = {"n": int(len(seg)), "start_min_us": float(st.min()), "start_max_us": float(st.max()),
+                     "end_max_us": float(en.max()), "dur_p50_us": float(np.median(dur)),
+                     "dur_mean_us": float(dur.mean()), "dur_max_us": float(dur.max()),
+                     "sms": int(len(np.unique(seg[:, 2] >> 32)))}
+    return out
