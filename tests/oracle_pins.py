@@ -340,9 +340,53 @@ def check_decode_step_driver(o):
         pred = r["pred_next"]
 
 
+def _brute_forced(v, K, n_sink, n_local):
+    """Forced sink/local blocks (sinks first, then newest local, within min(K, nb)), then
+    the unique completion whose members all rank before every non-member."""
+    nb = len(v)
+    keff = min(K, nb)
+    forced = [b for b in range(min(n_sink, nb))][:keff]
+    for i in range(n_local):
+        b = nb - 1 - i
+        if b < 0 or len(forced) >= keff:
+            break
+        if b not in forced:
+            forced.append(b)
+    rest = [b for b in range(nb) if b not in forced]
+    key = lambda b: (-v[b], b)
+    wins = [sub for sub in itertools.combinations(rest, keff - len(forced))
+            if all(key(a) < key(b) for a in sub for b in rest if b not in sub)]
+    assert len(wins) == 1
+    return sorted(forced + list(wins[0]))
+
+
+def check_selector_variants(o):
+    """Max-over-heads scores reduce to the sum for one head, bound every head's best
+    q.k and are exact with one token per block; forced sink/local selection matches
+    brute force and reduces to top-K with nothing forced."""
+    rng = np.random.default_rng(21)
+    k = _f(_grid_bits(rng, (512, 32)))
+    lo = np.stack([k[b * 64:(b + 1) * 64].min(0) for b in range(8)])
+    hi = np.stack([k[b * 64:(b + 1) * 64].max(0) for b in range(8)])
+    q1 = _f(_grid_bits(rng, (1, 32)))
+    assert np.array_equal(o.block_scores_max(q1, lo, hi), o.block_scores(q1, lo, hi))
+    q = _f(_grid_bits(rng, (4, 32)))
+    s = o.block_scores_max(q, lo, hi)
+    best = np.array([(q @ k[b * 64:(b + 1) * 64].T).max() for b in range(8)])
+    assert np.all(s >= best - 1e-12)
+    assert np.allclose(o.block_scores_max(q, k[:20], k[:20]), (q @ k[:20].T).max(0), atol=1e-12)
+    for seed in range(8):
+        r = np.random.default_rng(300 + seed)
+        nb, K = int(r.integers(1, 10)), int(r.integers(1, 5))
+        ns, nl = int(r.integers(0, 3)), int(r.integers(0, 3))
+        v = r.integers(0, 4, size=nb).astype(np.float64)
+        assert list(o.top_ranked_forced(v, K, ns, nl)) == _brute_forced(v, K, ns, nl)
+        assert np.array_equal(o.top_ranked_forced(v, K, 0, 0), o.top_ranked(v, K))
+
+
 ALL_CHECKS = [
     check_summaries_vs_numpy, check_bound_dominates_and_is_tight, check_grid_scores_exact,
     check_topk_bruteforce, check_ema_closed_form, check_predict_from_zero_state,
     check_attention_vs_sdpa, check_prr_invariance, check_merge_of_two_token_sets,
-    check_hand_examples, check_decode_step_driver,
+    check_hand_examples, check_decode_step_driver, check_selector_variants,
 ]

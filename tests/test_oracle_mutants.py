@@ -33,6 +33,9 @@ MUTANTS = [
      "if (contains(pred, npred, sel[i])) missed[nm++]"),
     ("partial_no_max_shift", "double p = exp(scale * dot_q_k(q, k + (size_t)t * d, d) - mm);",
      "double p = exp(scale * dot_q_k(q, k + (size_t)t * d, d));"),
+    ("variant_max_takes_min", "if (h == 0 || u > best) best = u;", "if (h == 0 || u < best) best = u;"),
+    ("variant_first_sink_skipped", "for (int b = 0; b < n_sink", "for (int b = 1; b < n_sink"),
+    ("variant_local_from_oldest", "int b = nb - 1 - i;", "int b = i;"),
 ]
 
 
