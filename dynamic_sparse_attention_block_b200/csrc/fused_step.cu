@@ -297,15 +297,6 @@ __global__ void __launch_bounds__(128, 3) fused_step_kernel(const __grid_constan
       bool dropped = sh[3] != 0;
       __syncthreads();
       if (blk >= 0 && blk < nb) {
-        // speculation has slack; selection is on the critical path.  Gate 1: wait until
-        // every selection tile has landed; gate 2: until every unit's S_t is published.
-        if (p.spec_gate != 0) {
-          if (p.spec_gate == 1) wait_geq(C.sel_loaded, static_cast<unsigned>(n_sel), C, p.status, sh);
-          if (p.spec_gate == 2) wait_geq(C.sel_finished, static_cast<unsigned>(U), C, p.status, sh);
-          if (tid == 0) sh[3] = (__ldcg(C.keepf + static_cast<size_t>(u) * p.P + j) == 1u) ? 1 : 0;
-          __syncthreads();
-          dropped = sh[3] != 0;
-        }
         const bool skip = dropped;
         if (!skip) {
           const size_t row0 = static_cast<size_t>(u) * p.G * p.P + j;

@@ -5,7 +5,6 @@
 
 #include <algorithm>
 #include <cmath>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <set>
@@ -89,15 +88,7 @@ DeviceInfo device_info() {
 
 // Blocks per selection CTA: about one CTA per SM over the whole (units x blocks) scan,
 // a multiple of 128 so every warp of the CTA streams at least one 32-block tile.
-// PRR_SELECT_CHUNK (environment, multiple of 32) overrides it for tuning.
 int select_chunk(int units, int maxnb, int sms) {
-  static int env = -1;
-  if (env < 0) {
-    const char* s = std::getenv("PRR_SELECT_CHUNK");
-    env = s ? std::atoi(s) : 0;
-    if (env < 0 || env % 32) env = 0;
-  }
-  if (env > 0) return env;
   const long long total = static_cast<long long>(units) * maxnb;
   long long c = (total + sms - 1) / sms;
   c = ((c + 127) / 128) * 128;
@@ -140,15 +131,6 @@ Params base_params(const prr_dims* d, void* ws) {
   // repair items per unit of the fused step: enough to spread a unit's misses over
   // many CTAs, few enough that empty items (most units miss little) stay cheap
   p.rep_items = std::min(p.K, std::max(4, (1024 + p.units - 1) / p.units));
-  {
-    static int gate = -1;  // PRR_SPEC_GATE in {0, 1, 2} overrides the speculation gate
-    if (gate < 0) {
-      const char* e = std::getenv("PRR_SPEC_GATE");
-      gate = (e && e[0] >= '0' && e[0] <= '2') ? e[0] - '0' : 0;
-    }
-    p.spec_gate = gate;
-  }
-
   return p;
 }
 

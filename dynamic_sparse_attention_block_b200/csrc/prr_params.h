@@ -49,7 +49,6 @@ struct Params {
   int fchunk_blocks; // blocks per SEL item
   int fused_region;  // bytes of the per-CTA shared-memory union
   int rep_items;     // REPAIR items per unit; item r repairs missed slots r, r + rep_items, ...
-  int spec_gate;     // speculative items wait: 0 no, 1 selection tiles landed, 2 all S_t published
   // caller buffers (any may be null when the kernel does not use it)
   const uint16_t* q;        // [B][Hq][d] bf16
   const uint16_t* kc;       // [B][Hkv][cap][d] bf16

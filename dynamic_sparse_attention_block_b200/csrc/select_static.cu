@@ -10,11 +10,17 @@
 // passes all inputs and outputs.
 //
 // The array is a file-scope __device__ variable, so every GPU that loads the library
-// holds it (PRR_SELECT_STATIC_SCRATCH_BYTES, about 4.3 MB) until the process exits.  Host code cannot use the array's
-// name as a device pointer: the device address is looked up once per device with
-// cudaGetSymbolAddress (on the first call made while that device is current) and then
-// passed to the kernel like any workspace pointer.
+// holds it (PRR_SELECT_STATIC_SCRATCH_BYTES, about 4.3 MB) until the process exits.
+// Host code cannot use the array's name as a device pointer: the device address is
+// looked up with cudaGetSymbolAddress on the first call made in a CUDA context (with
+// that context current) and then passed to the kernel like any workspace pointer.  The
+// address is cached per context, keyed by the context's process-unique id, so a
+// context created later on the same device (after cudaDeviceReset, say) looks the
+// address up again instead of writing through one that died with the old module.
+#include <cudaTypedefs.h>
+
 #include <cstring>
+#include <map>
 #include <mutex>
 
 #include "prr.h"
@@ -33,22 +39,56 @@ static_assert(kScratchBytes == PRR_SELECT_STATIC_SCRATCH_BYTES, "header and libr
 __device__ __align__(256) unsigned char g_select_scratch[kScratchBytes];
 
 std::mutex g_mu;
-void* g_addr[64] = {};
+std::map<unsigned long long, void*> g_addr;  // context id -> device address of the array
 
-// Device address of the scratch array on the current device (looked up once).
+// The driver's cuCtxGetCurrent and cuCtxGetId through the runtime's entry-point query
+// (the library does not link libcuda directly).
+struct CtxFns {
+  PFN_cuCtxGetCurrent_v4000 current = nullptr;
+  PFN_cuCtxGetId_v12000 id = nullptr;
+};
+
+CtxFns ctx_fns() {
+  static const CtxFns fns = [] {
+    CtxFns f;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+    ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.id = reinterpret_cast<PFN_cuCtxGetId_v12000>(ptr);
+    return f;
+  }();
+  return fns;
+}
+
+// Device address of the scratch array in the current context (looked up once per context).
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> g(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_select_scratch);
+  const CtxFns f = ctx_fns();
+  if (!f.current || !f.id) return cudaErrorDeviceUninitialized;
+  CUcontext ctx = nullptr;
+  void* fresh = nullptr;
+  if (f.current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  if (!ctx) {  // no context yet on this thread: the lookup itself brings up the device's
+    cudaError_t e = cudaGetSymbolAddress(&fresh, g_select_scratch);  // primary context
     if (e != cudaSuccess) return e;
-    g_addr[dev] = p;
+    if (f.current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
   }
-  *out = g_addr[dev];
+  unsigned long long id = 0;
+  if (f.id(ctx, &id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  std::lock_guard<std::mutex> g(g_mu);
+  auto it = g_addr.find(id);
+  if (it == g_addr.end()) {
+    if (!fresh) {
+      cudaError_t e = cudaGetSymbolAddress(&fresh, g_select_scratch);
+      if (e != cudaSuccess) return e;
+    }
+    it = g_addr.emplace(id, fresh).first;
+  }
+  *out = it->second;
   return cudaSuccess;
 }
 

@@ -287,9 +287,11 @@ prr_status prr_budget_choose(const double* sel_coef, const double* spec_coef, co
  *           (0 = ok, else one of PRR_DEV_*), written on `stream` after the kernel.
  * Returns PRR_ERR_CAPACITY, without enqueuing anything, when
  * B*Hkv*ceil(cap_tokens/bs) > PRR_SELECT_STATIC_MAX_BLOCKS.  Calls no cudaMalloc,
- * cudaFree or other allocating routine.  The first call on each device (made with
- * that device current) looks up the array's device address and keeps it; make that
- * first call before any stream capture.  Every call clears the status word and the
+ * cudaFree or other allocating routine.  The first call in each CUDA context (made
+ * with that context current) looks up the array's device address and keeps it for
+ * that context, so a context created later on the same device (for instance after
+ * cudaDeviceReset) gets the address again; make that first call before any stream
+ * capture.  Every call clears the status word and the
  * tickets on `stream` (the keys are always rewritten before use).  All calls share
  * the one array: calls whose work may overlap on the GPU (different streams without
  * ordering between them) race and give undefined results; order them on one stream. */

@@ -148,6 +148,21 @@ def check_ema_closed_form(o):
             assert np.allclose(e, closed, rtol=0, atol=1e-14), (alpha, t)
 
 
+def check_ema_rounding_fixed(o):
+    """The update rounds alpha*e and beta*ind separately, then their sum (no fused
+    multiply-add): the oracle reproduces, bit for bit, a trajectory derived with exact
+    rationals (tests/golden/ema_rounding.json, written by make_ema_rounding.py), which
+    a contracted update leaves at the step the fixture names."""
+    with open(os.path.join(GOLDEN, "ema_rounding.json")) as fh:
+        ex = json.load(fh)
+    e = np.zeros(ex["nb"])
+    for t, sel in enumerate(ex["selections"]):
+        e = o.ema_update(e, ex["nb"], np.array(sel, np.int32), ex["alpha"])
+        assert e[0].hex() == ex["e_block0_hex"][t], (t, e[0].hex())
+        assert e[1] == 0.0
+    assert ex["e_block0_hex"] != ex["contracted_block0_hex"]
+
+
 def check_predict_from_zero_state(o):
     """With no history all e = 0 and the tie rule predicts blocks 0..P-1."""
     for nb, P in [(65, 8), (5, 8), (513, 64)]:
@@ -386,7 +401,7 @@ def check_selector_variants(o):
 
 ALL_CHECKS = [
     check_summaries_vs_numpy, check_bound_dominates_and_is_tight, check_grid_scores_exact,
-    check_topk_bruteforce, check_ema_closed_form, check_predict_from_zero_state,
+    check_topk_bruteforce, check_ema_closed_form, check_ema_rounding_fixed, check_predict_from_zero_state,
     check_attention_vs_sdpa, check_prr_invariance, check_merge_of_two_token_sets,
     check_hand_examples, check_decode_step_driver, check_selector_variants,
 ]

@@ -5,10 +5,14 @@ compare them.  Inputs come only from ``workloads``; expected values come only fr
 Tolerances (fp32 attention on the GPU against fp64 on the CPU):
   selected sets, missed sets, keep masks, predicted sets, EMA state: bit-exact;
   out: max |gpu - oracle| <= 2e-3;  lse: |gpu - oracle| / |oracle| <= 1e-4.
-For Gaussian workloads a differing selected set is accepted when every differing
+For Gaussian workloads a differing selected set is accepted when it is a valid
+selection (ascending, distinct, in range, of size min(K, nb)) and every differing
 block's oracle score lies within 1e-5 * max(1, |s_K|) of the oracle's K-th score
-(the score-gap reading of the repair-sweep workload); such units are then not
-compared on out/lse.
+(the score-gap reading of the repair-sweep workload).  Several sets are then correct;
+the oracle continues from the GPU's accepted set, so the unit's missed set, keep
+mask, out, lse, EMA state and next prediction are still compared, against the
+oracle's values for that set.  Near ties must stay rare: at most
+max(NEAR_TIE_MIN, NEAR_TIE_FRAC * unit-steps) per run.
 """
 from __future__ import annotations
 
@@ -24,6 +28,8 @@ import workloads as W
 OUT_TOL = 2e-3
 LSE_RTOL = 1e-4
 GAP_RTOL = 1e-5
+NEAR_TIE_FRAC = 0.01
+NEAR_TIE_MIN = 2
 
 
 def f64(bits):
@@ -98,29 +104,62 @@ class Report:
     max_out_err: float = 0.0
     max_lse_rel: float = 0.0
     units_compared: int = 0
+    unit_steps: int = 0
     near_tie_units: int = 0
     messages: List[str] = field(default_factory=list)
 
     def fail(self, msg: str):
         self.messages.append(msg)
 
+    def near_tie_bound(self) -> int:
+        return max(NEAR_TIE_MIN, int(NEAR_TIE_FRAC * self.unit_steps))
+
+    def check_near_ties(self) -> None:
+        if self.near_tie_units > self.near_tie_bound():
+            self.fail(f"{self.near_tie_units} near-tie selections in {self.unit_steps} unit-steps "
+                      f"(bound {self.near_tie_bound()})")
+
+
+def accepted_selection(gpu_sel: np.ndarray, o_sel: np.ndarray, scores: np.ndarray,
+                       gaussian: bool) -> Optional[np.ndarray]:
+    """The set the comparison continues from, or None if the GPU's set is wrong.
+
+    Exact grids: only the oracle's set.  Gaussian scores: the GPU's set is also
+    accepted when it is a valid selection (strictly ascending, in range, as many blocks
+    as the oracle's) whose differences from the oracle's set all lie within the score
+    gap of the oracle's K-th score."""
+    g = np.asarray([int(x) for x in gpu_sel if x >= 0], np.int32)
+    r = np.asarray(o_sel, np.int32)
+    if np.array_equal(g, r):
+        return r
+    if not gaussian or len(g) != len(r):
+        return None
+    if np.any(np.diff(g) <= 0) or (len(g) and (g[0] < 0 or g[-1] >= len(scores))):
+        return None
+    if any(int(x) != -1 for x in np.asarray(gpu_sel)[len(g):]):
+        return None
+    kth = np.sort(scores)[::-1][len(r) - 1]
+    tol = GAP_RTOL * max(1.0, abs(kth))
+    diff = set(g.tolist()) ^ set(r.tolist())
+    if all(abs(scores[b] - kth) <= tol for b in diff):
+        return g
+    return None
+
 
 def check_selection(rep: Report, tag: str, gpu_sel: np.ndarray, o_sel: np.ndarray,
-                    scores: np.ndarray, K: int, gaussian: bool) -> bool:
-    """Returns True if sets are identical; records a failure unless a near tie allows it."""
-    g = [int(x) for x in gpu_sel if x >= 0]
-    r = [int(x) for x in o_sel]
-    if g == r:
-        return True
-    if gaussian and len(g) == len(r):
-        kth = np.sort(scores)[::-1][len(r) - 1]
-        tol = GAP_RTOL * max(1.0, abs(kth))
-        diff = set(g) ^ set(r)
-        if all(abs(scores[b] - kth) <= tol for b in diff):
-            rep.near_tie_units += 1
-            return False
-    rep.fail(f"{tag}: selected set differs: gpu={g} oracle={r}")
-    return False
+                    scores: np.ndarray, K: int, gaussian: bool) -> Optional[np.ndarray]:
+    """The selected set the oracle continues from for this unit: the oracle's set when
+    the GPU's equals it, the GPU's set when a Gaussian near tie makes it another
+    correct answer (counted in rep.near_tie_units), else None (a failure is recorded)."""
+    rep.unit_steps += 1
+    acc = accepted_selection(gpu_sel, o_sel, scores, gaussian)
+    if acc is None:
+        g = [int(x) for x in gpu_sel if x >= 0]
+        rep.fail(f"{tag}: selected set differs: gpu={g} oracle={list(map(int, o_sel))}")
+        return None
+    if not np.array_equal(acc, np.asarray(o_sel, np.int32)):
+        rep.near_tie_units += 1
+    return acc
 
 
 def compare_attention(rep: Report, tag: str, gpu_out: np.ndarray, gpu_lse: np.ndarray,

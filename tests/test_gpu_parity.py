@@ -10,7 +10,7 @@ import pytest
 
 import oracle as OR
 import workloads as W
-from tests.prr_harness import OUT_TOL, LSE_RTOL, f64, pad
+from tests.prr_harness import OUT_TOL, LSE_RTOL, accepted_selection, f64, pad
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -110,6 +110,7 @@ def test_select_topk(d, bs, G, K, P, n, gauss):
     keep = torch.zeros((B, Hkv, max(P, 1)), dtype=torch.uint8, device="cuda")
     pred = torch.from_numpy(pred_h).cuda()
     prr.prr_workspace_init(ws)
+    near_ties = 0
     for rep in range(2):  # second call checks that the tickets re-armed
         prr.prr_select_topk(dims, to_dev_bits(q), to_dev_bits(summ_h), seq, pred, sel, missed, nm, keep, ws)
         torch.cuda.synchronize()
@@ -118,12 +119,11 @@ def test_select_topk(d, bs, G, K, P, n, gauss):
         for b in range(B):
             for h in range(Hkv):
                 s = scores[(b, h)]
-                ref = o.top_ranked(s, K)
-                if gauss and list(g_sel[b, h][g_sel[b, h] >= 0]) != list(ref):
-                    kth = np.sort(s)[::-1][len(ref) - 1]
-                    diff = set(g_sel[b, h][g_sel[b, h] >= 0].tolist()) ^ set(ref.tolist())
-                    assert all(abs(s[x] - kth) <= 1e-5 * max(1, abs(kth)) for x in diff)
-                    continue
+                # Gaussian near ties: the GPU's set, if valid under the score gap, is the
+                # one missed and keep are checked against
+                ref = accepted_selection(g_sel[b, h], o.top_ranked(s, K), s, gauss)
+                assert ref is not None, (b, h, g_sel[b, h].tolist())
+                near_ties += int(not np.array_equal(ref, o.top_ranked(s, K)))
                 assert np.array_equal(g_sel[b, h], pad(ref, K)), (b, h)
                 pr = pred_h[b, h][pred_h[b, h] >= 0]
                 ref_missed, ref_keep = o.missed_keep(ref, pr)
@@ -131,6 +131,7 @@ def test_select_topk(d, bs, G, K, P, n, gauss):
                 assert g_nm[b, h] == len(ref_missed)
                 if P > 0:
                     assert np.array_equal(g_keep[b, h][:len(pr)], ref_keep)
+    assert near_ties <= 1, f"{near_ties} near-tie selections in {2 * B * Hkv} unit-calls"
 
 
 # ----------------------------------------------------------------------------- a4 EMA

@@ -22,6 +22,7 @@ MUTANTS = [
     ("tie_to_higher_index", "return ia < ib;", "return ia > ib;"),
     ("ema_alpha_beta_swapped", "double decayed = alpha * e[b];", "double decayed = beta * e[b];"),
     ("ema_no_decay", "double decayed = alpha * e[b];", "double decayed = e[b];"),
+    ("ema_contracted_fma", "e[b] = decayed + added;", "e[b] = fma(alpha, e[b], added);"),
     ("attention_scale_dropped", "double p = exp(scale * dot_q_k(q, k + (size_t)t * d, d) - m);",
      "double p = exp(dot_q_k(q, k + (size_t)t * d, d) - m);"),
     ("attention_tail_token_dropped",

@@ -1,16 +1,23 @@
 """prr_select_topk_static (fixed in-library scratch, no workspace) against
-prr_select_topk (caller workspace), through the C ABI.  Needs a B200; marked gpu.
+prr_select_topk (caller workspace) and against the fp64 oracle, through the C ABI.
+Needs a B200; marked gpu.
 
-Both run the same selection kernel, so the selected, missed and keep outputs must
-agree exactly, as the selection parity tests require against the oracle.  Two calls
-in a row with fresh inputs check that the shared scratch array, which keeps the
-previous call's contents, is re-armed correctly.  The file name sorts last so that
-pytest runs it after every other test; it also passes alone in a fresh process.
+Some callers cannot allocate device memory for a workspace (code inside another
+runtime's memory pool, hosts that forbid cudaMalloc once serving has started); the
+static entry point serves them from an array inside the library.  Both entry points
+run the same selection kernel, so the selected, missed and keep outputs must agree
+exactly, and on exact-grid inputs they must equal the oracle's top-K bit for bit.
+Two calls in a row with fresh inputs check that the shared scratch array, which keeps
+the previous call's contents, is re-armed correctly, also after a call that stopped
+early on a bad sequence length.  The file name sorts last so that pytest runs it
+after every other test; it also passes alone in a fresh process.
 """
 import numpy as np
 import pytest
 
+import oracle as OR
 import workloads as W
+from tests.prr_harness import f64, pad
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -68,6 +75,59 @@ def test_static_scratch_matches_workspace_entry(d, bs, G, K, P, n, gauss):
                 r, g = r[..., :P], g[..., :P]
             assert np.array_equal(r, g), f"call {call}: {name} differs"
         assert (ref[0] >= 0).sum().item() == B * Hkv * min(K, nb)
+        if not gauss:  # exact grid: the oracle's top-K, missed set and keep mask
+            _check_against_oracle(got, q, summ, pred_h, G, K, P, nb)
+
+
+def _check_against_oracle(got, q, summ, pred_h, G, K, P, nb):
+    o = OR.default()
+    qh = q.cpu().numpy().view(np.uint16)
+    sh = summ.cpu().numpy().view(np.uint16)
+    g_sel, g_missed, g_nm, g_keep = (x.cpu().numpy() for x in got)
+    B, Hkv = g_sel.shape[:2]
+    for b in range(B):
+        for h in range(Hkv):
+            s = o.block_scores(f64(qh[b, h * G:(h + 1) * G]), f64(sh[b, h, :nb, 0]), f64(sh[b, h, :nb, 1]))
+            ref = o.top_ranked(s, K)
+            assert np.array_equal(g_sel[b, h], pad(ref, K)), (b, h)
+            pr = pred_h[b, h][pred_h[b, h] >= 0]
+            ref_missed, ref_keep = o.missed_keep(ref, pr)
+            assert np.array_equal(g_missed[b, h], pad(ref_missed, K)) and g_nm[b, h] == len(ref_missed)
+            if P > 0:
+                assert np.array_equal(g_keep[b, h][:len(pr)], ref_keep)
+
+
+def test_static_scratch_recovers_after_bad_seq_len():
+    """A call whose sequence length is out of range reports status 1 (bad seq_len)
+    through the status word, with no fault, and leaves its units unfinished; the next
+    good call re-arms the shared array and matches prr_select_topk and the oracle."""
+    rng = np.random.default_rng(77)
+    B, Hkv, G, d, bs, K, P, n = 2, 2, 4, 128, 64, 16, 16, 5000
+    cap = n + 3
+    dims = prr.Dims(B=B, Hq=G * Hkv, Hkv=Hkv, d=d, bs=bs, cap_tokens=cap, K=K, P=P)
+    nb = -(-n // bs)
+    summ = _bits(rng, (B, Hkv, dims.maxnb, 2, d), False)
+    q = _bits(rng, (B, G * Hkv, d), False)
+    pred_h = np.full((B, Hkv, P), -1, np.int32)
+    for b in range(B):
+        for h in range(Hkv):
+            pred_h[b, h] = np.sort(rng.choice(nb, size=P, replace=False))
+    pred = torch.from_numpy(pred_h).cuda()
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    bad = torch.tensor([n, cap + 9], dtype=torch.int32, device="cuda")  # sequence 1 beyond the cache
+    prr.prr_select_topk_static(dims, q, summ, bad, pred, *_outputs(B, Hkv, K, P), status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1  # PRR_DEV_BAD_SEQ_LEN
+    seq = torch.full((B,), n, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(prr.prr_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    ref, got = _outputs(B, Hkv, K, P), _outputs(B, Hkv, K, P)
+    prr.prr_select_topk(dims, q, summ, seq, pred, *ref, ws)
+    prr.prr_select_topk_static(dims, q, summ, seq, pred, *got, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0 and prr.prr_get_device_status(ws) == 0
+    for r, g in zip(ref, got):
+        assert np.array_equal(r.cpu().numpy(), g.cpu().numpy())
+    _check_against_oracle(got, q, summ, pred_h, G, K, P, nb)
 
 
 def test_static_scratch_rejects_oversized_shapes():
