@@ -24,13 +24,19 @@ _i32 = ctypes.c_int32
 class PrrDims(ctypes.Structure):
     _fields_ = [("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("d", _i32), ("bs", _i32),
                 ("cap_tokens", _i32), ("K", _i32), ("P", _i32), ("alpha", ctypes.c_double),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("selector", _i32), ("n_sink", _i32), ("n_local", _i32),
+                ("pages", _i32), ("block_table", _c_void_p)]
+
+
+# block selectors (PRR_SELECT_* in include/prr.h)
+SELECTORS = {"group_sum": 0, "group_max": 1, "per_head": 2}
 
 
 class PrrStepBuffers(ctypes.Structure):
     _fields_ = [(n, _c_void_p) for n in (
         "q", "k_cache", "v_cache", "seq_lens", "summ", "ema", "pred", "pred_next", "sel",
-        "missed", "n_missed", "keep", "part_m", "part_l", "part_O", "out", "lse", "trace")]
+        "missed", "n_missed", "keep", "part_m", "part_l", "part_O", "out", "lse", "k_new", "v_new", "trace",
+        "stats")]
 
 
 STEP_EVENTS = ("fork", "sel_done", "spec_done", "join")
@@ -49,6 +55,9 @@ SYMBOLS = (
     "prr_ema_predict", "prr_speculate", "prr_repair_merge", "prr_decode_step",
     "prr_decode_step_fused", "prr_budget_fit", "prr_budget_choose", "prr_select_topk_static",
 )
+
+# mirrors PRR_WS_TEST_SKIP_SELECTION_OFFSET in include/prr.h
+WS_TEST_SKIP_SELECTION_OFFSET = 4
 
 # mirrors PRR_SELECT_STATIC_MAX_BLOCKS / PRR_SELECT_STATIC_SCRATCH_BYTES in include/prr.h
 SELECT_STATIC_MAX_BLOCKS = 1 << 20
@@ -125,14 +134,29 @@ class Dims:
     P: int
     alpha: float = 0.9
     scale: Optional[float] = None
+    selector: str = "group_sum"   # "group_sum", "group_max" or "per_head"
+    n_sink: int = 0               # forced first blocks
+    n_local: int = 0              # forced newest blocks
+    pages: int = 0                # paged KV pool size (0: contiguous caches)
+    block_table: Optional[int] = None  # device address of the int32 [B][maxnb] block table
 
     @property
     def G(self) -> int:
         return self.Hq // self.Hkv
 
     @property
+    def sel_heads(self) -> int:
+        """Selections per sequence: KV heads, or query heads under per-head selection."""
+        return self.Hq if self.selector == "per_head" else self.Hkv
+
+    @property
+    def group(self) -> int:
+        """Query heads one selection scores with (1 under per-head selection)."""
+        return 1 if self.selector == "per_head" else self.G
+
+    @property
     def units(self) -> int:
-        return self.B * self.Hkv
+        return self.B * self.sel_heads
 
     @property
     def maxnb(self) -> int:
@@ -141,7 +165,8 @@ class Dims:
     def c(self) -> PrrDims:
         sc = self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
         return PrrDims(self.B, self.Hq, self.Hkv, self.d, self.bs, self.cap_tokens, self.K,
-                       self.P, float(self.alpha), float(sc))
+                       self.P, float(self.alpha), float(sc), SELECTORS[self.selector], self.n_sink, self.n_local,
+                       self.pages, self.block_table)
 
 
 def _dims(d) -> PrrDims:

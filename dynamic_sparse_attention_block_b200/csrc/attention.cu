@@ -16,7 +16,7 @@ __global__ void __launch_bounds__(128) attn_block_kernel(const __grid_constant__
   const int tid = threadIdx.x;
   const int slot = blockIdx.x, u = blockIdx.y;
   const int G = p.G;
-  const int n = checked_len(p, u / p.Hkv);
+  const int n = checked_len(p, u / p.upb);
   const int nb = (n + BS - 1) / BS;
 
   int blk = -1;
@@ -45,10 +45,11 @@ __global__ void __launch_bounds__(128) attn_block_kernel(const __grid_constant__
   }
   if (!(blk >= 0 && blk < nb)) {  // a missed entry out of range: contribute nothing
     if (tid == 0) report(p.status, kDevBadMissed);
-    write_empty_partial(dst, G, D);
+    write_empty_partial(dst, G, D, cta_grp());
     return;
   }
   if (tid == 0) {
+    bump(p.stats, KIND == 0 ? kStatSpecAttended : kStatRepaired);
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
     mbar_init(&bars[0], 1);
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(128) attn_block_kernel(const __grid_constant__
     fence_barrier_init();
   }
   __syncthreads();
-  block_partial<D, BS>(p, &kmap, &vmap, u, blk, n, dst, smem, bars, 0u);
+  block_partial<D, BS>(p, &kmap, &vmap, u, blk, n, dst, smem, bars, 0u, cta_grp());
 }
 
 template <int D, int BS>

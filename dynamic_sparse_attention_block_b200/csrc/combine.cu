@@ -7,7 +7,7 @@ namespace prr {
 template <int D>
 __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(16) unsigned char smem[];
-  combine_head<D>(p, blockIdx.y, blockIdx.x, smem, [] { return true; });
+  combine_head<D>(p, blockIdx.y, blockIdx.x, smem, [] { return true; }, cta_grp());
 }
 
 cudaError_t launch_combine(const Params& p, cudaStream_t s, int priority) {

@@ -6,7 +6,7 @@ namespace prr {
 
 __global__ void __launch_bounds__(256) ema_predict_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(16) unsigned char smem[];
-  ema_unit(p, blockIdx.x, smem, [] { return true; });
+  ema_unit(p, blockIdx.x, smem, [] { return true; }, cta_grp());
 }
 
 cudaError_t launch_ema(const Params& p, cudaStream_t s, int priority) {

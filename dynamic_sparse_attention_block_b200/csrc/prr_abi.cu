@@ -31,15 +31,31 @@ bool dims_ok(const prr_dims* d) {
   if (d->cap_tokens < 1 || d->K < 1 || d->K > 128 || d->P < 0 || d->P > 128) return false;
   if (!(d->alpha >= 0.0 && d->alpha <= 1.0)) return false;
   if (!std::isfinite(d->scale)) return false;
-  const long long units = static_cast<long long>(d->B) * d->Hkv;
+  if (d->selector < PRR_SELECT_GROUP_SUM || d->selector > PRR_SELECT_PER_HEAD) return false;
+  if (d->n_sink < 0 || d->n_sink > (1 << 22) || d->n_local < 0 || d->n_local > (1 << 22)) return false;
+  if (d->pages < 0 || (d->pages > 0) != (d->block_table != nullptr)) return false;
+  if (static_cast<long long>(d->pages) * d->Hkv >= (1LL << 31)) return false;
+  const long long units = static_cast<long long>(d->B) * (d->selector == PRR_SELECT_PER_HEAD ? d->Hq : d->Hkv);
   if (units > 65535) return false;  // grid.y
   return true;
 }
 
+// Selection units and the query heads each one scores with.
+struct SelShape {
+  size_t units;
+  size_t G;
+};
+
+SelShape sel_shape(const prr_dims* d) {
+  if (d->selector == PRR_SELECT_PER_HEAD) return {static_cast<size_t>(d->B) * d->Hq, 1};
+  return {static_cast<size_t>(d->B) * d->Hkv, static_cast<size_t>(d->Hq / d->Hkv)};
+}
+
 WsLayout layout_for(const prr_dims* d) {
   WsLayout L = {};
-  const size_t units = static_cast<size_t>(d->B) * d->Hkv;
-  const size_t G = static_cast<size_t>(d->Hq / d->Hkv);
+  const SelShape sh = sel_shape(d);
+  const size_t units = sh.units;
+  const size_t G = sh.G;
   const size_t maxnb = static_cast<size_t>((d->cap_tokens + d->bs - 1) / d->bs);
   size_t off = 0;
   L.status = off;
@@ -57,7 +73,7 @@ WsLayout layout_for(const prr_dims* d) {
   L.rO = off;
   off = align256(off + 4 * units * G * d->K * d->d);
   L.ctl = off;
-  off = align256(off + 4 * 2 * (16 + 5 * units + units * static_cast<size_t>(d->P) + units * static_cast<size_t>(d->K)));
+  off = align256(off + 4 * 2 * fused_ctl_words_for(static_cast<int>(units), d->P, d->K, static_cast<int>(G)));
   L.total = off;
   return L;
 }
@@ -97,20 +113,34 @@ int select_chunk(int units, int maxnb, int sms) {
   return static_cast<int>(c);
 }
 
-Params base_params(const prr_dims* d, void* ws) {
+// Kernel parameters.  `kv_units`: the call works on KV heads whatever the selector
+// (summaries, appends); otherwise units follow the selector.
+Params base_params(const prr_dims* d, void* ws, bool kv_units = false) {
   Params p;
   std::memset(&p, 0, sizeof p);
   p.B = d->B;
   p.Hq = d->Hq;
   p.Hkv = d->Hkv;
   p.G = d->Hq / d->Hkv;
+  p.upb = d->Hkv;
+  p.kv_div = 1;
+  if (!kv_units && d->selector == PRR_SELECT_PER_HEAD) {
+    p.kv_div = p.G;
+    p.G = 1;
+    p.upb = d->Hq;
+  }
+  p.sel_max = d->selector == PRR_SELECT_GROUP_MAX && p.G > 1;
+  p.n_sink = d->n_sink;
+  p.n_local = d->n_local;
+  p.pages = d->pages;
+  p.table = d->block_table;
   p.d = d->d;
   p.bs = d->bs;
   p.cap = d->cap_tokens;
   p.K = d->K;
   p.P = d->P;
   p.maxnb = (d->cap_tokens + d->bs - 1) / d->bs;
-  p.units = d->B * d->Hkv;
+  p.units = d->B * p.upb;
   p.scale_log2 = static_cast<float>(static_cast<double>(d->scale) * 1.4426950408889634074);
   p.alpha = d->alpha;
   p.chunk_blocks = select_chunk(p.units, p.maxnb, device_info().sms);
@@ -127,10 +157,7 @@ Params base_params(const prr_dims* d, void* ws) {
     p.rO = reinterpret_cast<float*>(w + L.rO);
     p.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
   }
-  p.ctl_words = 16 + 5 * p.units + p.units * p.P + p.units * p.K;
-  // repair items per unit of the fused step: enough to spread a unit's misses over
-  // many CTAs, few enough that empty items (most units miss little) stay cheap
-  p.rep_items = std::min(p.K, std::max(4, (1024 + p.units - 1) / p.units));
+  p.ctl_words = static_cast<int>(fused_ctl_words_for(p.units, p.P, p.K, p.G));
   return p;
 }
 
@@ -158,15 +185,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D map over a KV cache [units][cap][d] bf16, box {64 channels, bs tokens, 1 unit},
-// 128-byte swizzle, zero fill outside the tensor.
+// 3-D map over a KV cache, box {64 channels, bs tokens, 1 slice}, 128-byte swizzle, zero
+// fill outside the tensor.  Contiguous caches [B*Hkv][cap][d]: a slice is one
+// (sequence, KV head) pair.  Paged pools [pages*Hkv][bs][d]: a slice is one (page, KV
+// head) tile.
 bool make_kv_map(CUtensorMap* map, const void* base, const prr_dims* d) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d->d), static_cast<cuuint64_t>(d->cap_tokens),
-                              static_cast<cuuint64_t>(d->B) * d->Hkv};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d->d) * 2,
-                                 static_cast<cuuint64_t>(d->d) * 2 * d->cap_tokens};
+  const bool paged = d->pages > 0;
+  const cuuint64_t rows = static_cast<cuuint64_t>(paged ? d->bs : d->cap_tokens);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d->d), rows,
+                              static_cast<cuuint64_t>(paged ? d->pages : d->B) * d->Hkv};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d->d) * 2, static_cast<cuuint64_t>(d->d) * 2 * rows};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(d->bs), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
@@ -243,7 +273,7 @@ prr_status prr_append_kv(const prr_dims* dims, const uint16_t* k_new, const uint
   if (!k_new || !v_new || !seq_lens || !k_cache || !v_cache || !ws) return PRR_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
     return PRR_ERR_INVALID_ARG;
-  Params p = base_params(dims, ws);
+  Params p = base_params(dims, ws, true);
   return cuda_status(launch_append_kv(p, k_new, v_new, k_cache, v_cache, seq_lens, stream));
 }
 
@@ -258,7 +288,7 @@ prr_status prr_update_summaries(const prr_dims* dims, const uint16_t* k_cache,
   if (!aligned16(k_cache) || !aligned16(summ)) return PRR_ERR_INVALID_ARG;
   if (max_range_tokens < 1 || max_range_tokens > dims->cap_tokens) return PRR_ERR_SHAPE;
   if (!tok_begin && max_range_tokens != 1) return PRR_ERR_SHAPE;
-  Params p = base_params(dims, ws);
+  Params p = base_params(dims, ws, true);
   p.kc = k_cache;
   p.summ = summ;
   p.seq_lens = seq_lens;
@@ -371,7 +401,8 @@ prr_status step_params(const prr_dims* dims, const prr_step_buffers* b, void* ws
   if (dims->P > 0 && (!b->pred || !b->pred_next || !b->keep || !b->part_m || !b->part_l || !b->part_O))
     return PRR_ERR_INVALID_ARG;
   if (dims->P > 0 && b->pred == b->pred_next) return PRR_ERR_INVALID_ARG;
-  if (!aligned16(b->k_cache) || !aligned16(b->v_cache) || !aligned16(b->summ) || !aligned16(b->out))
+  if (!aligned16(b->k_cache) || !aligned16(b->v_cache) || !aligned16(b->summ) || !aligned16(b->out) ||
+      !aligned16(b->q))
     return PRR_ERR_INVALID_ARG;
   if (b->part_O && !aligned16(b->part_O)) return PRR_ERR_INVALID_ARG;
   Params p = base_params(dims, ws);
@@ -393,7 +424,13 @@ prr_status step_params(const prr_dims* dims, const prr_step_buffers* b, void* ws
   p.out = b->out;
   p.lse = b->lse;
   p.append_summary = 1;
+  if ((b->k_new == nullptr) != (b->v_new == nullptr)) return PRR_ERR_INVALID_ARG;
+  if (b->k_new && (!aligned16(b->k_new) || !aligned16(b->v_new))) return PRR_ERR_INVALID_ARG;
+  p.k_new = b->k_new;
+  p.v_new = b->v_new;
+  p.append_kv = b->k_new ? 1 : 0;
   p.trace = b->trace;
+  p.stats = b->stats;
   *out = p;
   return PRR_OK;
 }
@@ -419,6 +456,11 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* b, void
     if ((x) != cudaSuccess) return PRR_ERR_CUDA; \
   } while (0)
   cudaStream_t A = select_stream, B = spec_stream;
+  if (p.append_kv) {  // the step's token first: the kernels below then see it in the cache
+    PRR_TRY(launch_append_kv(p, p.k_new, p.v_new, const_cast<uint16_t*>(p.kc), const_cast<uint16_t*>(p.vc),
+                             const_cast<int*>(p.seq_lens), A));
+    p.append_kv = 0;
+  }
   PRR_TRY(cudaEventRecord(ev->fork, A));
   PRR_TRY(cudaStreamWaitEvent(B, ev->fork, 0));
   // spec stream: speculation over Pred_t, independent of selection
@@ -455,11 +497,11 @@ prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* b
   Params p;
   const prr_status st = step_params(dims, b, ws, ws_bytes, &p);
   if (st != PRR_OK) return st;
-  if (fused_smem_bytes(p) > 227 * 1024) return PRR_ERR_SHAPE;
+  const DeviceInfo di = device_info();
+  if (fused_smem_bytes(p, di.sms) > 227 * 1024) return PRR_ERR_SHAPE;
   p.parity = step_parity;
   CUtensorMap km, vm;
   if (!make_kv_map(&km, b->k_cache, dims) || !make_kv_map(&vm, b->v_cache, dims)) return PRR_ERR_CUDA;
-  const DeviceInfo di = device_info();
   return cuda_status(launch_fused(p, km, vm, stream, di.prio_high, di.sms, nullptr));
 }
 

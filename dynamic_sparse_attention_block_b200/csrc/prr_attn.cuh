@@ -19,6 +19,10 @@
 // (an in-register 8x8 transpose).  P is split as bf16 hi + bf16 lo (two MMAs) so the
 // PV product keeps ~16 mantissa bits.  Four warps own disjoint token slices; their O^T
 // partial sums are added in shared memory.
+//
+// The copies and the arithmetic are separate steps (attn_issue, attn_compute): the
+// standalone kernels run both in one CTA; the fused step's producer warp issues the
+// copies into its ring while a consumer group computes an earlier block.
 #pragma once
 
 #include "prr_kernels.cuh"
@@ -29,7 +33,8 @@ template <int D, int BS>
 struct AttnTile {
   static constexpr int TILEB = BS * D * 2;  // one K or V tile
   static constexpr int REGB = BS * 128;     // one 64-channel swizzle region of a tile
-  static constexpr size_t bytes = 2 * static_cast<size_t>(TILEB) + 80 * 4;  // tiles + reductions
+  static constexpr int REDB = 80 * 4;       // cross-warp reductions
+  static constexpr size_t bytes = 2 * static_cast<size_t>(TILEB) + REDB;  // tiles + reductions
 };
 
 // Where one block's partial goes: m/l of head h at m[h*rstride], O at O[h*ostride].
@@ -41,59 +46,84 @@ struct PartialDst {
   size_t ostride;
 };
 
-__device__ __forceinline__ void write_empty_partial(const PartialDst& dst, int G, int D) {
-  for (int e = threadIdx.x; e < G * D; e += blockDim.x) dst.O[(e / D) * dst.ostride + (e % D)] = 0.f;
-  if (static_cast<int>(threadIdx.x) < G) {
-    dst.m[threadIdx.x * dst.rstride] = -INFINITY;
-    dst.l[threadIdx.x * dst.rstride] = 0.f;
+__device__ __forceinline__ void write_empty_partial(const PartialDst& dst, int G, int D, const Grp& g) {
+  for (int e = g.tid; e < G * D; e += g.nt) dst.O[(e / D) * dst.ostride + (e % D)] = 0.f;
+  if (g.tid < G) {
+    dst.m[g.tid * dst.rstride] = -INFINITY;
+    dst.l[g.tid * dst.rstride] = 0.f;
   }
 }
 
-// Partial of block `blk` of unit u (tokens below n).  Every thread of a 128-thread CTA
-// calls it.  `smem` is 1024-byte aligned with AttnTile::bytes free; bars[0], bars[1]
-// are initialised mbarriers (count 1) whose current phase parity is `phase` (both are
-// used once).  Returns false if a copy did not land in time (status word set).
+// One thread: start the K and V tiles of block `blk` of KV slice `slice` (the
+// tensor maps' third coordinate) towards sK / sV, completing on barK / barV.  Earlier
+// generic writes of this thread to the tiles are ordered before the copies.
 template <int D, int BS>
-__device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CUtensorMap* vmap, int u,
-                              int blk, int n, const PartialDst& dst, unsigned char* smem, uint64_t* bars,
-                              uint32_t phase) {
+__device__ __forceinline__ void attn_issue(const CUtensorMap* kmap, const CUtensorMap* vmap, int slice, int tok0,
+                                           unsigned char* sK, unsigned char* sV, uint64_t* barK, uint64_t* barV) {
   using L = AttnTile<D, BS>;
-  constexpr int TILEB = L::TILEB, REGB = L::REGB, NREG = D / 64;
+  constexpr int NREG = D / 64;
+  fence_proxy_async();
+  mbar_expect_tx(barK, L::TILEB);
+#pragma unroll
+  for (int r = 0; r < NREG; ++r) tma_load_3d(sK + r * L::REGB, kmap, barK, r * 64, tok0, slice);
+  mbar_expect_tx(barV, L::TILEB);
+#pragma unroll
+  for (int r = 0; r < NREG; ++r) tma_load_3d(sV + r * L::REGB, vmap, barV, r * 64, tok0, slice);
+}
+
+// Write one token row (d bf16, 16-byte aligned, global) into row r of a staged tile in
+// its 128-byte swizzled position.  The group's first D/8 threads each move 16 bytes.
+template <int D, int BS>
+__device__ __forceinline__ void tile_put_row(unsigned char* tile, int r, const uint16_t* row, const Grp& g) {
+  using L = AttnTile<D, BS>;
+  if (g.tid < D / 8) {
+    const int rr = g.tid >> 3, c16 = g.tid & 7;
+    *reinterpret_cast<uint4*>(tile + rr * L::REGB + r * 128 + ((c16 ^ (r & 7)) << 4)) =
+        *reinterpret_cast<const uint4*>(row + g.tid * 8);
+  }
+}
+
+// Partial of the block whose K/V tiles are (being) staged in sK / sV, tokens below n of
+// block `blk`.  Every thread of a 128-thread group calls it.  `q` points at the G query
+// rows of the unit ([G][D] bf16, global or shared).  barK / barV are the tiles'
+// mbarriers, waited on with parity `phase` (bounded).  When `patch_k` is not null, the
+// token n-1 (which lies in this block) is taken from patch_k / patch_v instead of the
+// staged tiles (the caller has not written it to the cache yet).  `red` is 80 floats of
+// shared scratch.  Returns false if a copy did not land in time (status word set).
+template <int D, int BS>
+__device__ bool attn_compute(const Params& p, const uint16_t* q, int blk, int n, const PartialDst& dst,
+                             unsigned char* sK, unsigned char* sV, float* red, uint64_t* barK, uint64_t* barV,
+                             uint32_t phase, const Grp& grp, const uint16_t* patch_k = nullptr,
+                             const uint16_t* patch_v = nullptr) {
+  using L = AttnTile<D, BS>;
+  constexpr int REGB = L::REGB, NREG = D / 64;
   constexpr int MTW = BS / 64;  // 16-token m-tiles per warp (4 warps)
   constexpr int KS = D / 16;    // k-steps of QK^T == 16-channel tiles of PV
-  unsigned char* sK = smem;
-  unsigned char* sV = smem + TILEB;
-  float* red = reinterpret_cast<float*>(smem + 2 * TILEB);  // [0,32) max, [32,64) sum, [64,72) m, [72,80) l
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
   const int G = p.G;
-
-  if (tid == 0) {
-    fence_proxy_async();  // earlier generic writes to these tiles precede the copies
-    mbar_expect_tx(&bars[0], TILEB);
-#pragma unroll
-    for (int r = 0; r < NREG; ++r) tma_load_3d(sK + r * REGB, kmap, &bars[0], r * 64, blk * BS, u);
-    mbar_expect_tx(&bars[1], TILEB);
-#pragma unroll
-    for (int r = 0; r < NREG; ++r) tma_load_3d(sV + r * REGB, vmap, &bars[1], r * 64, blk * BS, u);
-  }
 
   // Q^T fragments (B operand of the score product): lane (g, t) holds head g,
   // channels 16ks + 2t, +1 and 16ks + 2t + 8, +9.  Heads >= G are zero.
   const int g = lane >> 2, t = lane & 3;
   uint32_t qf[KS][2];
   {
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(u) * G + (g < G ? g : 0)) * D);
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(q + (g < G ? g : 0) * D);
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
-      qf[ks][0] = g < G ? __ldg(qrow + ks * 8 + t) : 0u;
-      qf[ks][1] = g < G ? __ldg(qrow + ks * 8 + 4 + t) : 0u;
+      qf[ks][0] = g < G ? qrow[ks * 8 + t] : 0u;
+      qf[ks][1] = g < G ? qrow[ks * 8 + 4 + t] : 0u;
     }
   }
 
   const int nv = min(BS, n - blk * BS);  // valid tokens of this block
-  if (!__syncthreads_and(mbar_wait(&bars[0], phase, p.status))) {
-    if (tid == 0) mbar_wait(&bars[1], phase, p.status);  // let the V copy land (bounded)
+  const int prow = n - 1 - blk * BS;      // row of token n-1 when a patch is given
+  if (!gsync_and(grp, mbar_wait(barK, phase, p.status))) {
+    if (tid == 0) mbar_wait(barV, phase, p.status);  // let the V copy land (bounded)
     return false;
+  }
+  if (patch_k) {
+    tile_put_row<D, BS>(sK, prow, patch_k, grp);
+    gsync(grp);
   }
 
   // ---- S^T = K Q^T on the tensor cores
@@ -136,7 +166,7 @@ __device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CU
     red[warp * 8 + 2 * t] = mx0;
     red[warp * 8 + 2 * t + 1] = mx1;
   }
-  __syncthreads();
+  gsync(grp);
   float m0 = red[2 * t], m1 = red[2 * t + 1];
 #pragma unroll
   for (int w = 1; w < 4; ++w) {
@@ -171,16 +201,17 @@ __device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CU
     red[32 + warp * 8 + 2 * t + 1] = ls1;
   }
 
-  if (!__syncthreads_and(mbar_wait(&bars[1], phase, p.status))) return false;
+  if (!gsync_and(grp, mbar_wait(barV, phase, p.status))) return false;
   if (nv < BS) {  // tokens past the end of the sequence: zero V so 0 * V stays 0
     uint4* v4 = reinterpret_cast<uint4*>(sV);
     const int rows = BS - nv;
-    for (int i = tid; i < rows * NREG * 8; i += blockDim.x) {
+    for (int i = tid; i < rows * NREG * 8; i += grp.nt) {
       const int r = nv + i / (NREG * 8), rem = i % (NREG * 8);
       v4[((rem >> 3) * REGB + r * 128) / 16 + (rem & 7)] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  __syncthreads();
+  if (patch_v) tile_put_row<D, BS>(sV, prow, patch_v, grp);
+  gsync(grp);
   if (warp == 0 && g == 0) {
     float l0 = 0.f, l1 = 0.f;
 #pragma unroll
@@ -212,7 +243,8 @@ __device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CU
       mma_16816(oacc[dt], a, bl[mi][0], bl[mi][1]);
     }
   }
-  // per-warp O^T into the (dead) K tile: redO[warp][h][c ^ 4h], conflict-free
+  // per-warp O^T into the (dead) K tile: redO[warp][h][c ^ 4h], conflict-free (every
+  // warp passed a group barrier after its last K-tile read)
   float* redO = reinterpret_cast<float*>(sK);
 #pragma unroll
   for (int dt = 0; dt < KS; ++dt) {
@@ -222,9 +254,9 @@ __device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CU
     redO[(warp * 8 + 2 * t) * D + ((c0 + 8) ^ (8 * t))] = oacc[dt][2];
     redO[(warp * 8 + 2 * t + 1) * D + ((c0 + 8) ^ (8 * t + 4))] = oacc[dt][3];
   }
-  __syncthreads();
+  gsync(grp);
   constexpr int C4 = D / 4;
-  for (int e = tid; e < G * C4; e += blockDim.x) {
+  for (int e = tid; e < G * C4; e += grp.nt) {
     const int h = e / C4, c4 = e % C4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -243,6 +275,25 @@ __device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CU
   }
   fence_proxy_async();  // this thread's generic writes to the tiles precede later copies
   return true;
+}
+
+// Both steps in one group (standalone kernels): partial of block `blk` of unit u.
+// `smem` is 1024-byte aligned with AttnTile::bytes free; bars[0], bars[1] are
+// initialised mbarriers (count 1) whose current phase parity is `phase`.
+template <int D, int BS>
+__device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CUtensorMap* vmap, int u,
+                              int blk, int n, const PartialDst& dst, unsigned char* smem, uint64_t* bars,
+                              uint32_t phase, const Grp& grp) {
+  using L = AttnTile<D, BS>;
+  unsigned char* sK = smem;
+  unsigned char* sV = smem + L::TILEB;
+  if (grp.tid == 0) {
+    int tok0;
+    const int slice = kv_tile(p, u / p.kv_div, blk, &tok0);
+    attn_issue<D, BS>(kmap, vmap, slice, tok0, sK, sV, &bars[0], &bars[1]);
+  }
+  return attn_compute<D, BS>(p, p.q + static_cast<size_t>(u) * p.G * D, blk, n, dst, sK, sV,
+                             reinterpret_cast<float*>(smem + 2 * L::TILEB), &bars[0], &bars[1], phase, grp);
 }
 
 }  // namespace prr

@@ -17,6 +17,16 @@ enum : int {
   kDevBadRange = 5,        // summary update range outside [0, cap_tokens]
 };
 
+// Counters of prr_step_buffers::stats.
+enum : int {
+  kStatTieMasks = 0,
+  kStatKeySearch = 1,
+  kStatTakeAll = 2,
+  kStatSpecAttended = 3,
+  kStatSpecSkipped = 4,
+  kStatRepaired = 5,
+};
+
 // A bounded wait gives up after this long (one second).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
@@ -29,16 +39,26 @@ struct WsLayout {
   size_t rm;         // float [units*G][K] repair partial max (base-2 logits)
   size_t rl;         // float [units*G][K] repair partial sum
   size_t rO;         // float [units*G][K][d] repair partial numerator
-  size_t ctl;        // uint32 [2][16 + 5*units + units*(P + K)] control words of the fused step
+  size_t ctl;        // uint32 [2][ctl_words] control words of the fused step (see fused_step.cu)
   size_t total;
 };
 
 struct Params {
-  // shape
+  // shape.  A unit is one selection: a (sequence, KV head) pair, or a (sequence, query
+  // head) pair under per-head selection.  G = query heads per unit (1 per head).
   int B, Hq, Hkv, G, d, bs, cap, K, P, maxnb, units;
+  int upb;      // units per sequence: sequence of unit u = u / upb
+  int kv_div;   // KV (and summary) slice of unit u = u / kv_div
+  int sel_max;  // block score = largest per-head bound of the group instead of their sum
+  int n_sink;   // forced first blocks
+  int n_local;  // forced newest blocks
+  // paged KV: pools [pages][Hkv][bs][d], table [B][maxnb] block -> page (null: contiguous)
+  int pages;
+  const int* table;
   float scale_log2;  // softmax scale * log2(e): logits are handled in base 2
   double alpha;      // EMA decay
-  int append_summary;  // selection also folds token seq_lens[b]-1 into its block summary
+  int append_summary;  // selection also folds token n-1 into its block summary
+  int append_kv;       // the fused step appends k_new/v_new itself: n = seq_lens[b] + 1
   // selection geometry
   int chunk_blocks;  // blocks per selection CTA (multiple of 32)
   int nchunks;       // selection CTAs per unit
@@ -46,11 +66,15 @@ struct Params {
   int parity;        // which copy of the control words this launch uses
   int ctl_words;     // words per copy
   int fchunks;       // SEL items per unit
-  int fchunk_blocks; // blocks per SEL item
-  int fused_region;  // bytes of the per-CTA shared-memory union
-  int rep_items;     // REPAIR items per unit; item r repairs missed slots r, r + rep_items, ...
+  int fchunk_blocks; // blocks per SEL item (multiple of 32, at most 128)
+  int fslots;        // item slots of the shared-memory ring
+  int fslot_bytes;   // bytes of one slot's main area (tiles, summary rows or task scratch)
+  int fbatch;        // main tickets a producer claims per atomic
+  int rq_cap;        // ready-queue entries per control-word copy
   // caller buffers (any may be null when the kernel does not use it)
   const uint16_t* q;        // [B][Hq][d] bf16
+  const uint16_t* k_new;    // [B][Hkv][d] bf16 token appended by the fused step (append_kv)
+  const uint16_t* v_new;    // [B][Hkv][d] bf16
   const uint16_t* kc;       // [B][Hkv][cap][d] bf16
   const uint16_t* vc;       // [B][Hkv][cap][d] bf16
   const int* seq_lens;      // [B]
@@ -77,6 +101,7 @@ struct Params {
   float* rO;
   unsigned* ctl;
   unsigned long long* trace;  // optional: per fused item {start ns, end ns, sm, item}
+  unsigned long long* stats;  // optional: step counters (see prr_step_buffers::stats)
   // summary update range (null: append of token seq_lens[b]-1)
   const int* tok_begin;
   const int* tok_end;

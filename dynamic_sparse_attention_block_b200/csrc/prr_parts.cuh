@@ -15,7 +15,7 @@ namespace prr {
 __device__ unsigned long long g_phase[2][4096][8];
 #define PRR_PHASE(kind, u, k) \
   do {                        \
-    if (threadIdx.x == 0 && (u) < 4096) g_phase[kind][u][k] = global_ns(); \
+    if ((threadIdx.x & 127) == 0 && (u) < 4096) g_phase[kind][u][k] = global_ns(); \
   } while (0)
 #else
 #define PRR_PHASE(kind, u, k) \
@@ -30,17 +30,17 @@ __device__ unsigned long long g_phase[2][4096][8];
 // would wait one memory round trip per element.
 constexpr int kBatch = 16;
 
-__device__ __forceinline__ void load_words_cg(uint32_t* dst, const uint32_t* src, int n) {
-  for (int base = 0; base < n; base += kBatch * static_cast<int>(blockDim.x)) {
+__device__ __forceinline__ void load_words_cg(uint32_t* dst, const uint32_t* src, int n, const Grp& g) {
+  for (int base = 0; base < n; base += kBatch * g.nt) {
     uint32_t v[kBatch];
 #pragma unroll
     for (int q = 0; q < kBatch; ++q) {
-      const int i = base + q * blockDim.x + threadIdx.x;
+      const int i = base + q * g.nt + g.tid;
       v[q] = i < n ? __ldcg(src + i) : 0u;
     }
 #pragma unroll
     for (int q = 0; q < kBatch; ++q) {
-      const int i = base + q * blockDim.x + threadIdx.x;
+      const int i = base + q * g.nt + g.tid;
       if (i < n) dst[i] = v[q];
     }
   }
@@ -56,16 +56,17 @@ __device__ __forceinline__ void load_words_cg(uint32_t* dst, const uint32_t* src
 // 2^24 units of 1/64, so the fp32 score is exact in any order.
 
 // Coefficients of the [min | max] summary row, element e in chunk e/8: positions 0-3
-// in lo[chunk], 4-7 in hi[chunk].  All threads call; synchronise before use.
+// in lo[chunk], 4-7 in hi[chunk], from the G query rows qg ([G][D] bf16, global or
+// shared).  The group's threads call; synchronise before use.
 template <int D>
-__device__ __forceinline__ void load_group_coef(const Params& p, int u, float4* lo4, float4* hi4) {
+__device__ __forceinline__ void load_group_coef(const Params& p, const uint16_t* qg, float4* lo4, float4* hi4,
+                                                const Grp& g) {
   float* lo = reinterpret_cast<float*>(lo4);
   float* hi = reinterpret_cast<float*>(hi4);
-  const uint16_t* qg = p.q + static_cast<size_t>(u) * p.G * D;
-  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+  for (int c = g.tid; c < D; c += g.nt) {
     uint16_t qv[8];  // G <= 8: every head's load in flight before the first is used
 #pragma unroll
-    for (int h = 0; h < 8; ++h) qv[h] = h < p.G ? __ldg(qg + h * D + c) : static_cast<uint16_t>(0);
+    for (int h = 0; h < 8; ++h) qv[h] = h < p.G ? qg[h * D + c] : static_cast<uint16_t>(0);
     float neg = 0.f, pos = 0.f;
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
@@ -103,6 +104,93 @@ __device__ __forceinline__ float score_summary_row(const unsigned char* row, con
     acc = fmaf(z.w, bf16_hi(w.w), acc);
   }
   return acc;
+}
+
+// Selector variant (group max): the block score is the LARGEST of the group's per-head
+// bounds, max_h sum_c max(q_hc*min_bc, q_hc*max_bc).  Per head the bound is again one
+// dot product, with coefficients min(q_hc, 0) against the min row and max(q_hc, 0)
+// against the max row; coef holds G such sets, set h at coef + 2*C*h (lo parts) and
+// coef + 2*C*h + C (hi parts), C = 4D/16 chunks, laid out as in load_group_coef.
+template <int D>
+__device__ __forceinline__ void load_head_coef(const Params& p, const uint16_t* qg, float4* coef, const Grp& g) {
+  constexpr int C = 4 * D / 16;
+  for (int i = g.tid; i < p.G * D; i += g.nt) {
+    const int h = i / D, c = i % D;
+    const float x = __uint_as_float(static_cast<uint32_t>(qg[h * D + c]) << 16);
+    float* lo = reinterpret_cast<float*>(coef + 2 * C * h);
+    float* hi = reinterpret_cast<float*>(coef + 2 * C * h + C);
+    const int e0 = c, e1 = D + c;  // min part, max part
+    ((e0 & 7) < 4 ? lo[(e0 >> 3) * 4 + (e0 & 3)] : hi[(e0 >> 3) * 4 + (e0 & 3)]) = fminf(x, 0.f);
+    ((e1 & 7) < 4 ? lo[(e1 >> 3) * 4 + (e1 & 3)] : hi[(e1 >> 3) * 4 + (e1 & 3)]) = fmaxf(x, 0.f);
+  }
+}
+
+// Largest per-head bound of one block (row in shared memory); every head's products of
+// a 16-byte chunk reuse the chunk's unpacked values.  Exact on the dyadic grid.
+template <int D>
+__device__ __forceinline__ float score_summary_row_max(const unsigned char* row, const float4* coef, int G,
+                                                       int lane) {
+  constexpr int C = 4 * D / 16;
+  float acc[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) acc[h] = 0.f;
+#pragma unroll 2
+  for (int i = 0; i < C; ++i) {
+    const int cc = (i + lane) & (C - 1);
+    const uint4 w = *reinterpret_cast<const uint4*>(row + cc * 16);
+    const float x0 = bf16_lo(w.x), x1 = bf16_hi(w.x), x2 = bf16_lo(w.y), x3 = bf16_hi(w.y);
+    const float x4 = bf16_lo(w.z), x5 = bf16_hi(w.z), x6 = bf16_lo(w.w), x7 = bf16_hi(w.w);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if (h < G) {
+        const float4 a = coef[2 * C * h + cc], z = coef[2 * C * h + C + cc];
+        float s = acc[h];
+        s = fmaf(a.x, x0, s);
+        s = fmaf(a.y, x1, s);
+        s = fmaf(a.z, x2, s);
+        s = fmaf(a.w, x3, s);
+        s = fmaf(z.x, x4, s);
+        s = fmaf(z.y, x5, s);
+        s = fmaf(z.z, x6, s);
+        s = fmaf(z.w, x7, s);
+        acc[h] = s;
+      }
+    }
+  }
+  float m = acc[0];
+#pragma unroll
+  for (int h = 1; h < 8; ++h)
+    if (h < G) m = fmaxf(m, acc[h]);
+  return m;
+}
+
+// Bytes of the scoring coefficients: one set for the group sum, G sets for the max.
+__host__ __device__ constexpr size_t coef_bytes(int D, int sets) { return static_cast<size_t>(sets) * 2 * (4 * D / 16) * 16; }
+
+// Both variants: coefficients for unit u's query rows qg (group-synchronise before use).
+template <int D>
+__device__ __forceinline__ void load_coef(const Params& p, const uint16_t* qg, float4* coef, const Grp& g) {
+  if (p.sel_max) {
+    load_head_coef<D>(p, qg, coef, g);
+  } else {
+    load_group_coef<D>(p, qg, coef, coef + (4 * D / 16), g);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ float score_row(const Params& p, const unsigned char* row, const float4* coef, int lane) {
+  if (p.sel_max) return score_summary_row_max<D>(row, coef, p.G, lane);
+  return score_summary_row<D>(row, coef, coef + (4 * D / 16), lane);
+}
+
+// Ranking key of block b (of nb) with score s: forced sink blocks rank above
+// everything, then forced local blocks, newest first, then every other block by its
+// score (orderable keys of finite scores stay below 0xFF800001).  Top-K over these keys
+// takes the sinks first, then the newest local blocks, then the best of the rest.
+__device__ __forceinline__ uint32_t block_key(const Params& p, int b, int nb, float s) {
+  if (b < p.n_sink) return 0xFFFFFFFFu;
+  if (b >= nb - p.n_local) return 0xFFFFFFFEu - static_cast<uint32_t>(nb - 1 - b);
+  return orderable(s);
 }
 
 // Fold the appended token's key row (newk, d bf16 in shared memory) into the summary
@@ -164,6 +252,7 @@ __device__ __forceinline__ void write_group_summary(const Params& p, int u, int 
 struct FinishOut {
   int p_active;  // active predicted slots
   int n_missed;
+  int path;      // kStatTakeAll, kStatTieMasks or kStatKeySearch
 };
 
 __host__ __device__ constexpr size_t finish_scratch_bytes(int maxnb) {
@@ -175,9 +264,9 @@ __host__ __device__ constexpr size_t finish_scratch_bytes(int maxnb) {
 // rdesc [K], per missed slot, block + 1 (kNoRepair past the last missed block).
 constexpr unsigned kNoRepair = 0xFFFFFFFFu;
 
-__device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsigned char* scratch,
+__device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsigned char* scratch, const Grp& grp,
                                           unsigned* keepf = nullptr, unsigned* rdesc = nullptr) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, NT = blockDim.x;
+  const int tid = grp.tid, warp = tid >> 5, lane = tid & 31, NT = grp.nt;
   const int W = (p.maxnb + 31) / 32;
   int* spred = reinterpret_cast<int*>(scratch + 256 * 4);  // [128]
   int* misc = spred + 128;                                 // counts, T, n_gt
@@ -199,12 +288,12 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
     for (int g = tid; g < Wn; g += NT) gs[g] = __ldcg(src + g);
   }
   if (!take_all && nb <= kEagerKeys) {  // with the summaries: no second round trip if no tie
-    load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb);
+    load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb, grp);
     have_keys = true;
   }
   for (int i = tid; i < W; i += NT) bm_pred[i] = 0u;
   if (tid < 16) misc[tid] = 0;
-  __syncthreads();
+  gsync(grp);
   PRR_PHASE(0, u, 1);
   int active_local = 0;
   for (int j = tid; j < p.P; j += NT) {
@@ -231,7 +320,7 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
     }
     mx = __reduce_max_sync(kFull, mx);
     if (lane == 0) atomicMax(&ms[6], mx);
-    __syncthreads();
+    gsync(grp);
     const uint32_t gmax = ms[6];
     int ce = 0;
     if (use_gs) {
@@ -241,15 +330,15 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
     }
     ce = __reduce_add_sync(kFull, ce);
     if (lane == 0 && ce) atomicAdd(&misc[7], ce);
-    __syncthreads();
+    gsync(grp);
     if (misc[7] >= keff) {
       T = gmax;
       tie_masks = use_gs;
     } else {
       if (!have_keys && !take_all) {
-        load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb);
+        load_words_cg(skeys, p.keys + static_cast<size_t>(u) * p.maxnb, nb, grp);
         have_keys = true;
-        __syncthreads();
+        gsync(grp);
       }
       if (warp == 0) {  // T bit by bit; every candidate count is one warp reduction
         uint32_t t, gt;
@@ -325,7 +414,7 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
           misc[9] = static_cast<int>(gt);
         }
       }
-      __syncthreads();
+      gsync(grp);
       T = ms[8];
       n_gt = misc[9];
     }
@@ -364,7 +453,7 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
         base += __shfl_sync(kFull, inc, 31);
       }
     }
-    __syncthreads();
+    gsync(grp);
   } else {
     select_bitmap(
         nb, take_all ? 0 : keff - n_gt,
@@ -373,7 +462,7 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
           const uint32_t kv = skeys[i];
           return kv > T ? 1 : (kv == T ? 0 : -1);
         },
-        bm_sel, bm_eq);
+        bm_sel, bm_eq, grp);
   }
   // three warps in parallel: selected list, missed list, keep mask
   int nm = 0;
@@ -385,10 +474,13 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
     nm = warp_emit_bitmap(bm_sel, bm_pred, Wn, p.missed + static_cast<size_t>(u) * p.K, p.K, [&](int pos, int b) {
       if (rdesc) rdesc[pos] = static_cast<unsigned>(b) + 1u;
       if (p.kc && p.vc) {
-        const int rows = min(p.bs, p.cap - b * p.bs);
-        const size_t off = (static_cast<size_t>(u) * p.cap + static_cast<size_t>(b) * p.bs) * p.d;
-        prefetch_l2(p.kc + off, static_cast<uint32_t>(rows) * p.d * 2);
-        prefetch_l2(p.vc + off, static_cast<uint32_t>(rows) * p.d * 2);
+        const int rows = p.table ? p.bs : min(p.bs, p.cap - b * p.bs);
+        const long long r0 = kv_row(p, u / p.kv_div, b * p.bs);  // a block's rows are contiguous
+        if (r0 >= 0) {
+          const size_t off = static_cast<size_t>(r0) * p.d;
+          prefetch_l2(p.kc + off, static_cast<uint32_t>(rows) * p.d * 2);
+          prefetch_l2(p.vc + off, static_cast<uint32_t>(rows) * p.d * 2);
+        }
       }
     });
     if (rdesc)
@@ -406,12 +498,14 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
   }
   // active predicted slots (CTA sum of the per-thread counts)
   if (tid == 0) misc[3] = 0;
-  __syncthreads();
+  gsync(grp);
   if (active_local) atomicAdd(&misc[3], active_local);
-  __syncthreads();
+  gsync(grp);
   PRR_PHASE(0, u, 4);
   PRR_PHASE(0, u, 5);
-  return FinishOut{misc[3], misc[2]};
+  const int path = take_all ? kStatTakeAll : (tie_masks ? kStatTieMasks : kStatKeySearch);
+  if (tid == 0 && keff > 0) bump(p.stats, path);
+  return FinishOut{misc[3], misc[2], path};
 }
 
 // ------------------------------------------------------------------ EMA predictor
@@ -443,7 +537,7 @@ __host__ __device__ constexpr size_t ema_scratch_bytes(int maxnb) {
 // Every thread of the CTA calls it.  wait_sel() (CTA-wide) returns once S_t may be read,
 // false to give up; the state copy is started before it, so its latency is hidden.
 template <typename WaitFn>
-__device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, WaitFn wait_sel) {
+__device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, WaitFn wait_sel, const Grp& grp) {
   const int W = (p.maxnb + 31) / 32;
   unsigned* hist = reinterpret_cast<unsigned*>(scratch);  // 16-byte aligned
   int* misc = reinterpret_cast<int*>(hist + 256);         // [4] candidates, [5] |S_t|
@@ -454,13 +548,13 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, 
   unsigned* bsel = bm + W;                                    // predicted set
   unsigned* beq = bsel + W;
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = grp.tid, warp = tid >> 5, lane = tid & 31, NT = grp.nt;
   PRR_PHASE(1, u, 0);
   double* e = p.ema + static_cast<size_t>(u) * p.maxnb;
   const bool update = p.sel != nullptr;
   // state copy up to the allocation (entries >= nb are unused), before any wait
-  for (int i = tid; i < p.maxnb; i += blockDim.x) cp_async_8(ev + i, e + i);
-  for (int i = tid; i < W; i += blockDim.x) {
+  for (int i = tid; i < p.maxnb; i += NT) cp_async_8(ev + i, e + i);
+  for (int i = tid; i < W; i += NT) {
     bm[i] = 0u;
     bsel[i] = 0u;
   }
@@ -470,32 +564,32 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, 
   }
   if (!wait_sel()) {
     cp_async_wait_all();
-    __syncthreads();
+    gsync(grp);
     return;
   }
   int sv = -1;
   if (update && tid < p.K) sv = __ldcg(p.sel + static_cast<size_t>(u) * p.K + tid);
-  const int n = checked_len(p, u / p.Hkv);
+  const int n = checked_len(p, u / p.upb, grp);
   const int nb = (n + p.bs - 1) / p.bs;
   const int Wn = (nb + 31) / 32;
   const int peff = min(p.P, nb);
   cp_async_wait_all();
-  __syncthreads();
+  gsync(grp);
   bool ranked = false;
   if (update) {
-    for (int i = tid; i < p.K; i += blockDim.x) {
+    for (int i = tid; i < p.K; i += NT) {
       const int v = i == tid ? sv : __ldcg(p.sel + static_cast<size_t>(u) * p.K + i);
       if (v >= 0 && v < nb) atomicOr(&bm[v >> 5], 1u << (v & 31));
     }
-    __syncthreads();
+    gsync(grp);
     int nsel = 0;
-    for (int i = tid; i < Wn; i += blockDim.x) nsel += __popc(bm[i]);
+    for (int i = tid; i < Wn; i += NT) nsel += __popc(bm[i]);
     if (nsel) atomicAdd(&misc[5], nsel);
-    __syncthreads();
+    gsync(grp);
     const bool filter = peff > 0 && peff < nb && peff <= misc[5];
     const double alpha = p.alpha;
     const double beta = __dsub_rn(1.0, alpha);
-    for (int base = 0; base < nb; base += blockDim.x) {  // warp-uniform trip count
+    for (int base = 0; base < nb; base += NT) {  // warp-uniform trip count
       const int i = base + tid;
       bool cand = false;
       unsigned long long bits = 0ull;
@@ -519,11 +613,11 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, 
         }
       }
     }
-    __syncthreads();
+    gsync(grp);
     const int cnt = misc[4];
     if (filter && cnt <= kEmaCand) {
       ranked = true;
-      for (int c = tid; c < cnt; c += blockDim.x) {
+      for (int c = tid; c < cnt; c += NT) {
         const unsigned long long kc = ckey[c];
         const int ic = cidx[c];
         int rank = 0;
@@ -533,14 +627,14 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, 
         }
         if (rank < peff) atomicOr(&bsel[ic >> 5], 1u << (ic & 31));
       }
-      __syncthreads();
+      gsync(grp);
     }
   }
   PRR_PHASE(1, u, 1);
 
   int* out = p.pred_next + static_cast<size_t>(u) * p.P;
   if (peff <= 0) {
-    for (int j = tid; j < p.P; j += blockDim.x) out[j] = -1;
+    for (int j = tid; j < p.P; j += NT) out[j] = -1;
     return;
   }
   auto hi = [&](int i) { return static_cast<uint32_t>(static_cast<unsigned long long>(__double_as_longlong(ev[i])) >> 32); };
@@ -548,15 +642,15 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, 
   if (ranked) {
     // bsel holds the predicted set
   } else if (peff >= nb) {
-    select_bitmap(nb, 0, [&](int) { return 1; }, bsel, beq);
+    select_bitmap(nb, 0, [&](int) { return 1; }, bsel, beq, grp);
   } else {
     int gt_hi = 0, gt_lo = 0;
-    const uint32_t Thi = radix_kth_largest(nb, peff, hi, [&](int) { return true; }, hist, misc, &gt_hi);
+    const uint32_t Thi = radix_kth_largest(nb, peff, hi, [&](int) { return true; }, hist, misc, &gt_hi, grp);
     PRR_PHASE(1, u, 2);
     const int need = peff - gt_hi;  // taken from the entries tied on the high word
     // low word among the entries tied on the high word (no pass at all when they agree)
     const uint32_t Tlo = radix_kth_largest(
-        nb, need, lo, [&](int i) { return hi(i) == Thi; }, hist, misc, &gt_lo);
+        nb, need, lo, [&](int i) { return hi(i) == Thi; }, hist, misc, &gt_lo, grp);
     PRR_PHASE(1, u, 3);
     select_bitmap(
         nb, need - gt_lo,
@@ -566,10 +660,10 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, 
           const uint32_t l = lo(i);
           return l > Tlo ? 1 : (l == Tlo ? 0 : -1);
         },
-        bsel, beq);
+        bsel, beq, grp);
   }
   if (warp == 0) warp_emit_bitmap(bsel, nullptr, Wn, out, p.P);
-  __syncthreads();
+  gsync(grp);
   PRR_PHASE(1, u, 4);
 }
 
@@ -624,7 +718,8 @@ __device__ __forceinline__ void fold_batch(WarpState& st, const float (&m)[B], c
 }
 
 template <int D, typename WaitFn>
-__device__ void combine_head(const Params& p, int u, int h, unsigned char* scratch, WaitFn wait_repair) {
+__device__ void combine_head(const Params& p, int u, int h, unsigned char* scratch, WaitFn wait_repair,
+                             const Grp& grp) {
   constexpr int C4 = D / 4;
   constexpr int B = 8;  // slots per batch and warp: 8 float4 loads in flight per lane
   const int P = p.P, K = p.K;
@@ -635,20 +730,20 @@ __device__ void combine_head(const Params& p, int u, int h, unsigned char* scrat
   int* count = reinterpret_cast<int*>(red + 8);
   float4* part = reinterpret_cast<float4*>((reinterpret_cast<uintptr_t>(red + 16) + 15) &
                                            ~static_cast<uintptr_t>(15));  // [4][C4]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
   const size_t row = static_cast<size_t>(u) * p.G + h;
   const bool col = lane < C4;
   WarpState st{-INFINITY, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
 
   // ---- speculative slots: flags and statistics in one round trip, then numerators
-  for (int j = tid; j < P; j += blockDim.x) {
+  for (int j = tid; j < P; j += grp.nt) {
     const bool act = __ldcg(p.keep + static_cast<size_t>(u) * P + j) != 0;
     const float m = __ldcg(p.pm + row * P + j);
     const float l = __ldcg(p.pl + row * P + j);
     km[j] = act ? m : -INFINITY;
     kl[j] = act ? l : 0.f;
   }
-  __syncthreads();
+  gsync(grp);
   if (warp == 0) {
     int cnt = 0;
     for (int base = 0; base < P; base += 32) {
@@ -660,7 +755,7 @@ __device__ void combine_head(const Params& p, int u, int h, unsigned char* scrat
     }
     if (lane == 0) count[0] = cnt;
   }
-  __syncthreads();
+  gsync(grp);
   const int ns = count[0];
   for (int s0 = warp; s0 < ns; s0 += 4 * B) {
     float m[B], l[B];
@@ -709,7 +804,7 @@ __device__ void combine_head(const Params& p, int u, int h, unsigned char* scrat
     red[4 + warp] = st.l;
   }
   if (col) part[warp * C4 + lane] = st.o;
-  __syncthreads();
+  gsync(grp);
   const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
   float L = 0.f, f[4];
 #pragma unroll
@@ -735,7 +830,7 @@ __device__ void combine_head(const Params& p, int u, int h, unsigned char* scrat
     reinterpret_cast<float4*>(p.out + row * D)[tid] = o;
   }
   if (tid == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
-  __syncthreads();
+  gsync(grp);
 }
 
 }  // namespace prr

@@ -9,10 +9,12 @@
 // 32 entries); trimming the ties and writing a set in ascending index order take one
 // warp, popcounts and a shuffle prefix sum.  These routines run once per step on the
 // critical path, so they use few barriers and no CTA-wide scans.  Every thread of the
-// CTA must call the functions that contain __syncthreads (marked "CTA").
+// group must call the functions that synchronise it (marked "Group"; see Grp).
 #pragma once
 
 #include <cstdint>
+
+#include "prr_device.cuh"
 
 namespace prr {
 
@@ -29,15 +31,15 @@ __device__ __forceinline__ int warp_inclusive_sum(int v) {
   return v;
 }
 
-// CTA.  k-th largest key (1 <= k <= number of members) among entries i < n with
+// Group.  k-th largest key (1 <= k <= number of members) among entries i < n with
 // member(i).  Returns T; *n_gt = number of members with key > T.  `hist`: 256
 // unsigned of 16-byte aligned shared scratch; `bc`: 2 ints of shared scratch.
 // Leading bytes shared by every member key (one min/max reduction) need no pass, so
 // scores in a narrow range usually take two or three passes.
 template <typename KeyFn, typename MemberFn>
 __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, unsigned* hist, int* bc,
-                                      int* n_gt) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, NT = blockDim.x, nw = NT >> 5;
+                                      int* n_gt, const Grp& grp) {
+  const int tid = grp.tid, lane = tid & 31, warp = tid >> 5, NT = grp.nt, nw = NT >> 5;
   unsigned kmin = 0xFFFFFFFFu, kmax = 0u;
   for (int i = tid; i < n; i += NT) {
     if (member(i)) {
@@ -52,13 +54,13 @@ __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, 
     hist[warp] = kmin;
     hist[32 + warp] = kmax;
   }
-  __syncthreads();
+  gsync(grp);
   unsigned gmin = 0xFFFFFFFFu, gmax = 0u;
   for (int w = 0; w < nw; ++w) {
     gmin = min(gmin, hist[w]);
     gmax = max(gmax, hist[32 + w]);
   }
-  __syncthreads();  // hist is reused below
+  gsync(grp);  // hist is reused below
   if (gmin == gmax) {  // all member keys equal
     *n_gt = 0;
     return gmin;
@@ -70,7 +72,7 @@ __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, 
 #pragma unroll 1
   for (int shift = 24 - 8 * skip; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += NT) hist[i] = 0u;
-    __syncthreads();
+    gsync(grp);
     for (int base = 0; base < n; base += NT) {  // warp-uniform trip count
       const int i = base + tid;
       unsigned dg = 0u;
@@ -91,7 +93,7 @@ __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, 
         else if (act && dg != d0) atomicAdd(&hist[dg], 1u);
       }
     }
-    __syncthreads();
+    gsync(grp);
     if (warp == 0) {
       // lane l owns bins 8l..8l+7; suffix sums run from the top bin down
       const uint4 a = reinterpret_cast<const uint4*>(hist)[2 * lane];
@@ -121,7 +123,7 @@ __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, 
         }
       }
     }
-    __syncthreads();
+    gsync(grp);
     const uint32_t dsel = static_cast<uint32_t>(bc[0]);
     const int above = bc[1];
     above_total += above;
@@ -129,17 +131,17 @@ __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, 
     prefix |= dsel << shift;
     pmask |= 0xFFu << shift;
   }
-  __syncthreads();  // bc / hist reusable
+  gsync(grp);  // bc / hist reusable
   *n_gt = above_total;
   return prefix;
 }
 
-// CTA.  Bitmap `bm` (ceil(n/32) words) of the entries with cmp(i) > 0 plus the
+// Group.  Bitmap `bm` (ceil(n/32) words) of the entries with cmp(i) > 0 plus the
 // `take_equal` lowest-index entries with cmp(i) == 0 (cmp(i) < 0: not selected).
 // `eq` is scratch of the same size.  On return bm is complete and visible to all.
 template <typename CmpFn>
-__device__ void select_bitmap(int n, int take_equal, CmpFn cmp, unsigned* bm, unsigned* eq) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+__device__ void select_bitmap(int n, int take_equal, CmpFn cmp, unsigned* bm, unsigned* eq, const Grp& grp) {
+  const int lane = grp.tid & 31, warp = grp.tid >> 5, nw = grp.nt >> 5;
   const int W = (n + 31) / 32;
   for (int wd = warp; wd < W; wd += nw) {
     const int i = wd * 32 + lane;
@@ -151,7 +153,7 @@ __device__ void select_bitmap(int n, int take_equal, CmpFn cmp, unsigned* bm, un
       eq[wd] = e;
     }
   }
-  __syncthreads();
+  gsync(grp);
   if (warp == 0 && take_equal > 0) {  // the first take_equal tie bits, in index order
     int base = 0;
     for (int w0 = 0; w0 < W; w0 += 32) {
@@ -177,7 +179,7 @@ __device__ void select_bitmap(int n, int take_equal, CmpFn cmp, unsigned* bm, un
       if (base >= take_equal) break;
     }
   }
-  __syncthreads();
+  gsync(grp);
 }
 
 // One warp.  Write the set bits of bm[0..W) (optionally masked by ~exclude) as

@@ -103,7 +103,9 @@ extern "C" prr_status prr_select_topk_static(const prr_dims* dims, const uint16_
   if (dims->P > 0 && (!pred || !keep)) return PRR_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(summ) & 15u) != 0) return PRR_ERR_INVALID_ARG;
 
-  const int units = dims->B * dims->Hkv;
+  const bool per_head = dims->selector == PRR_SELECT_PER_HEAD;
+  const int upb = per_head ? dims->Hq : dims->Hkv;  // selection units per sequence
+  const int units = dims->B * upb;
   const int maxnb = (dims->cap_tokens + dims->bs - 1) / dims->bs;
   if (static_cast<long long>(units) * maxnb > PRR_SELECT_STATIC_MAX_BLOCKS) return PRR_ERR_CAPACITY;
 
@@ -120,7 +122,14 @@ extern "C" prr_status prr_select_topk_static(const prr_dims* dims, const uint16_
   p.B = dims->B;
   p.Hq = dims->Hq;
   p.Hkv = dims->Hkv;
-  p.G = dims->Hq / dims->Hkv;
+  p.G = per_head ? 1 : dims->Hq / dims->Hkv;
+  p.upb = upb;
+  p.kv_div = per_head ? dims->Hq / dims->Hkv : 1;
+  p.sel_max = dims->selector == PRR_SELECT_GROUP_MAX && p.G > 1;
+  p.n_sink = dims->n_sink;
+  p.n_local = dims->n_local;
+  p.pages = dims->pages;
+  p.table = dims->block_table;
   p.d = dims->d;
   p.bs = dims->bs;
   p.cap = dims->cap_tokens;

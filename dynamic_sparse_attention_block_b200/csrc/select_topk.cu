@@ -31,7 +31,7 @@ struct SelectSmem {
   static constexpr int C = ROWB / 16;       // 16-byte chunks per summary row
   static constexpr size_t stages = 0;       // 4 streaming warps x 2 stages
   static constexpr size_t coef = stages + 8 * STAGE;
-  static constexpr size_t newk = coef + 2 * C * 16;  // appended key row (d bf16)
+  static constexpr size_t newk = coef + 8 * 2 * C * 16;  // coefficients: up to 8 per-head sets; then the key row
   static constexpr size_t bars = newk + 2 * D;
   static constexpr size_t misc = bars + 8 * 8;
   static constexpr size_t fin = misc + 16 * 4;  // finisher scratch
@@ -41,28 +41,30 @@ struct SelectSmem {
 template <int D>
 __global__ void __launch_bounds__(256, 1) select_topk_kernel(const __grid_constant__ Params p) {
   using L = SelectSmem<D>;
-  constexpr int ROWB = L::ROWB, STAGE = L::STAGE, C = L::C;
+  constexpr int ROWB = L::ROWB, STAGE = L::STAGE;
   extern __shared__ __align__(1024) unsigned char smem[];
-  float4* coef_lo = reinterpret_cast<float4*>(smem + L::coef);
-  float4* coef_hi = coef_lo + C;
+  float4* coef = reinterpret_cast<float4*>(smem + L::coef);
   uint16_t* newk = reinterpret_cast<uint16_t*>(smem + L::newk);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars);
   int* misc = reinterpret_cast<int*>(smem + L::misc);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x, u = blockIdx.y;
-  const int n = checked_len(p, u / p.Hkv);
+  const int n = checked_len(p, u / p.upb);
   const int nb = (n + p.bs - 1) / p.bs;
   const int c0 = chunk * p.chunk_blocks;
   const int cnt = max(0, min(p.chunk_blocks, nb - c0));
   const int nrounds = (cnt + 31) / 32;
   const int tail = n > 0 ? (n - 1) / p.bs : -1;
   const bool own_tail = p.append_summary && tail >= c0 && tail < c0 + cnt;
-  uint16_t* summ_unit = p.summ + static_cast<size_t>(u) * p.maxnb * 2 * D;
+  const int kvu = u / p.kv_div;  // KV slice (several units share it under per-head selection)
+  uint16_t* summ_unit = p.summ + static_cast<size_t>(kvu) * p.maxnb * 2 * D;
 
-  load_group_coef<D>(p, u, coef_lo, coef_hi);
-  if (own_tail) {  // the appended token's key row
-    const uint16_t* krow = p.kc + (static_cast<size_t>(u) * p.cap + (n - 1)) * D;
+  const Grp grp = cta_grp();
+  load_coef<D>(p, p.q + static_cast<size_t>(u) * p.G * D, coef, grp);
+  const long long trow = own_tail ? kv_row(p, kvu, n - 1) : -1;
+  if (own_tail && trow >= 0) {  // the appended token's key row
+    const uint16_t* krow = p.kc + static_cast<size_t>(trow) * D;
     for (int c = tid; c < D / 8; c += blockDim.x)
       reinterpret_cast<uint4*>(newk)[c] = __ldg(reinterpret_cast<const uint4*>(krow) + c);
   }
@@ -105,12 +107,12 @@ __global__ void __launch_bounds__(256, 1) select_topk_kernel(const __grid_consta
       const int first = c0 + r * 32;
       const int rows = min(32, cnt - r * 32);
       unsigned char* tile = ring + s * STAGE;
-      if (own_tail && tail >= first && tail < first + rows)
+      if (own_tail && trow >= 0 && tail >= first && tail < first + rows)
         fold_tail_row<D>(reinterpret_cast<uint32_t*>(tile + (tail - first) * ROWB), newk, ((n - 1) % p.bs) == 0,
                          reinterpret_cast<uint32_t*>(summ_unit + static_cast<size_t>(tail) * 2 * D), lane);
       uint32_t key = 0u;
       if (lane < rows) {
-        key = orderable(score_summary_row<D>(tile + lane * ROWB, coef_lo, coef_hi, lane));
+        key = block_key(p, first + lane, nb, score_row<D>(p, tile + lane * ROWB, coef, lane));
         keys_out[first + lane] = key;
       }
       write_group_summary(p, u, first / 32, key, lane < rows);
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(256, 1) select_topk_kernel(const __grid_consta
   if (!misc[0]) return;
   __threadfence();
   if (tid == 0) p.sel_cnt[u] = 0u;
-  select_finish(p, u, nb, smem + L::fin);
+  select_finish(p, u, nb, smem + L::fin, grp);
 }
 
 size_t select_smem_bytes(int d, int maxnb) {

@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(128) update_summaries_kernel(const __grid_cons
   const bool fresh = (lo_t == t0);  // range covers the block from its first token
 
   const int c = threadIdx.x % C, rg = threadIdx.x / C;
+  const long long r0 = kv_row(p, u, t0);  // the block's rows are contiguous in the cache
+  if (r0 < 0) return;
   // +inf / -inf bf16 pairs as the identities of min / max
   __nv_bfloat162 mn[4], mx[4];
   const __nv_bfloat162 pinf = __halves2bfloat162(__ushort_as_bfloat16(0x7F80), __ushort_as_bfloat16(0x7F80));
@@ -49,9 +51,9 @@ __global__ void __launch_bounds__(128) update_summaries_kernel(const __grid_cons
 #pragma unroll
   for (int i = 0; i < 4; ++i) { mn[i] = pinf; mx[i] = ninf; }
 
-  const uint16_t* base = p.kc + (static_cast<size_t>(u) * p.cap) * D + c * 8;
+  const uint16_t* base = p.kc + static_cast<size_t>(r0) * D + c * 8;
   for (int t = lo_t + rg; t < hi_t; t += RG) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t) * D));
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(t - t0) * D));
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -99,13 +101,15 @@ __global__ void __launch_bounds__(128) append_kv_kernel(const Params p, const ui
                                                         uint16_t* vc, int* seq_lens) {
   const int b = blockIdx.x;
   const int pos = seq_lens[b];
-  const bool ok = pos >= 0 && pos < p.cap;
+  bool ok = pos >= 0 && pos < p.cap;
   if (ok) {
     constexpr int C = D / 8;
     for (int i = threadIdx.x; i < p.Hkv * C; i += blockDim.x) {
       const int h = i / C, c = i % C;
+      const long long row = kv_row(p, b * p.Hkv + h, pos);
+      if (row < 0) continue;  // bad block-table entry (reported)
       const size_t src = (static_cast<size_t>(b) * p.Hkv + h) * D + c * 8;
-      const size_t dst = ((static_cast<size_t>(b) * p.Hkv + h) * p.cap + pos) * D + c * 8;
+      const size_t dst = static_cast<size_t>(row) * D + c * 8;
       *reinterpret_cast<uint4*>(kc + dst) = *reinterpret_cast<const uint4*>(k_new + src);
       *reinterpret_cast<uint4*>(vc + dst) = *reinterpret_cast<const uint4*>(v_new + src);
     }

@@ -6,6 +6,7 @@ libprr_b200.so through the C ABI.
 """
 from __future__ import annotations
 
+import dataclasses
 from typing import Optional
 
 import torch
@@ -18,31 +19,46 @@ class PRRDecoder:
     """Caller-owned state of the PRR decode step (PRR abstract / method summary: EMA
     predictor, speculative attention overlapped with selection, repair + LSE merge).
 
-    Buffers (row-major):  k_cache/v_cache [B][Hkv][cap][d] bf16, seq_lens [B] int32,
-    summ [B][Hkv][maxnb][2][d] bf16, ema [B][Hkv][maxnb] fp64, pred double buffer
-    [2][B][Hkv][P] int32, sel/missed [B][Hkv][K], n_missed [B][Hkv], keep [B][Hkv][P],
+    Buffers (row-major), with S = selections per sequence (Hkv; Hq under per-head
+    selection):  k_cache/v_cache [B][Hkv][cap][d] bf16, seq_lens [B] int32,
+    summ [B][Hkv][maxnb][2][d] bf16, ema [B][S][maxnb] fp64, pred double buffer
+    [2][B][S][P] int32, sel/missed [B][S][K], n_missed [B][S], keep [B][S][P],
     speculative partials [B][Hq][P](+[d]) fp32, out [B][Hq][d] fp32, lse [B][Hq] fp32.
     """
 
-    def __init__(self, dims: Dims, device: Optional[torch.device] = None):
+    def __init__(self, dims: Dims, device: Optional[torch.device] = None,
+                 block_table: Optional[torch.Tensor] = None):
+        """dims.pages > 0 makes the KV cache a paged pool [pages][Hkv][bs][d];
+        `block_table` (int32 [B][maxnb], page of block j of sequence b) then defaults to
+        block j of sequence b in page b*maxnb + j."""
         if not torch.cuda.is_available():
             raise RuntimeError("PRRDecoder needs a CUDA device")
         _abi.load()
-        self.dims = dims
         self.device = torch.device(device or "cuda")
         dev = self.device
         B, Hq, Hkv, d, cap, K, P = dims.B, dims.Hq, dims.Hkv, dims.d, dims.cap_tokens, dims.K, dims.P
+        S = dims.sel_heads  # selections per sequence (per-unit arrays are [B][S][...])
         maxnb = dims.maxnb
-        self.k_cache = torch.zeros((B, Hkv, cap, d), dtype=torch.bfloat16, device=dev)
-        self.v_cache = torch.zeros((B, Hkv, cap, d), dtype=torch.bfloat16, device=dev)
+        self.block_table = None
+        if dims.pages > 0:
+            if block_table is None:
+                block_table = torch.arange(B * maxnb, dtype=torch.int32).view(B, maxnb)
+            self.block_table = block_table.to(device=dev, dtype=torch.int32).contiguous()
+            self.table_host = self.block_table.cpu().numpy()
+            dims = dataclasses.replace(dims, block_table=self.block_table.data_ptr())
+            self.k_cache = torch.zeros((dims.pages, Hkv, dims.bs, d), dtype=torch.bfloat16, device=dev)
+        else:
+            self.k_cache = torch.zeros((B, Hkv, cap, d), dtype=torch.bfloat16, device=dev)
+        self.dims = dims
+        self.v_cache = torch.zeros_like(self.k_cache)
         self.seq_lens = torch.zeros((B,), dtype=torch.int32, device=dev)
         self.summ = torch.zeros((B, Hkv, maxnb, 2, d), dtype=torch.bfloat16, device=dev)
-        self.ema = torch.zeros((B, Hkv, maxnb), dtype=torch.float64, device=dev)
-        self.pred_buf = torch.full((2, B, Hkv, max(P, 1)), -1, dtype=torch.int32, device=dev)
-        self.sel = torch.full((B, Hkv, K), -1, dtype=torch.int32, device=dev)
-        self.missed = torch.full((B, Hkv, K), -1, dtype=torch.int32, device=dev)
-        self.n_missed = torch.zeros((B, Hkv), dtype=torch.int32, device=dev)
-        self.keep = torch.zeros((B, Hkv, max(P, 1)), dtype=torch.uint8, device=dev)
+        self.ema = torch.zeros((B, S, maxnb), dtype=torch.float64, device=dev)
+        self.pred_buf = torch.full((2, B, S, max(P, 1)), -1, dtype=torch.int32, device=dev)
+        self.sel = torch.full((B, S, K), -1, dtype=torch.int32, device=dev)
+        self.missed = torch.full((B, S, K), -1, dtype=torch.int32, device=dev)
+        self.n_missed = torch.zeros((B, S), dtype=torch.int32, device=dev)
+        self.keep = torch.zeros((B, S, max(P, 1)), dtype=torch.uint8, device=dev)
         self.part_m = torch.zeros((B, Hq, max(P, 1)), dtype=torch.float32, device=dev)
         self.part_l = torch.zeros((B, Hq, max(P, 1)), dtype=torch.float32, device=dev)
         self.part_O = torch.zeros((B, Hq, max(P, 1), d), dtype=torch.float32, device=dev)
@@ -70,6 +86,7 @@ class PRRDecoder:
         self.parity = 0  # which pred buffer holds Pred_t
         self.fused_parity = 0  # control-word copy of the next fused launch
         self.trace = None      # optional per-item timeline of fused launches (enable_trace)
+        self.stats = None      # optional step counters (enable_stats)
 
     # ------------------------------------------------------------------ views
     @property
@@ -80,7 +97,9 @@ class PRRDecoder:
     def pred_next(self) -> torch.Tensor:
         return self.pred_buf[1 - self.parity]
 
-    def buffers(self, parity: Optional[int] = None) -> _abi.PrrStepBuffers:
+    def buffers(self, parity: Optional[int] = None, append: bool = False) -> _abi.PrrStepBuffers:
+        """Step buffers; with `append` the step also appends the token held in the
+        decoder's k_new / v_new buffers (it then advances seq_lens itself)."""
         par = self.parity if parity is None else parity
         b = _abi.PrrStepBuffers()
         b.q, b.k_cache, b.v_cache = self.q.data_ptr(), self.k_cache.data_ptr(), self.v_cache.data_ptr()
@@ -90,7 +109,10 @@ class PRRDecoder:
         b.keep = self.keep.data_ptr()
         b.part_m, b.part_l, b.part_O = self.part_m.data_ptr(), self.part_l.data_ptr(), self.part_O.data_ptr()
         b.out, b.lse = self.out.data_ptr(), self.lse.data_ptr()
+        if append:
+            b.k_new, b.v_new = self.k_new.data_ptr(), self.v_new.data_ptr()
         b.trace = self.trace.data_ptr() if self.trace is not None else None
+        b.stats = self.stats.data_ptr() if self.stats is not None else None
         return b
 
     def events(self, timing: Optional[dict] = None) -> _abi.PrrStepEvents:
@@ -105,13 +127,15 @@ class PRRDecoder:
             setattr(e, name, ev.cuda_event)
         return e
 
-    def fused_items(self) -> dict:
-        """Work-item counts of one fused launch, in queue order."""
+    def fused_items(self, sms: Optional[int] = None) -> dict:
+        """Trace records of one fused launch, in record order: the main work (selection
+        chunks, then speculative slots) and the task records (repairs, predictor
+        updates and merges, in the order they were queued)."""
         d = self.dims
-        rep = min(d.K, max(4, -(-1024 // d.units)))
-        chunk = min(128, max(32, -(-(-(-d.units * d.maxnb // 512)) // 32) * 32))
-        return {"sel": d.units * -(-d.maxnb // chunk), "fin": d.units, "ema": d.units,
-                "spec": d.units * d.P, "repair": d.units * rep, "combine": d.units * d.G}
+        sms = sms or torch.cuda.get_device_properties(self.device).multi_processor_count
+        chunk = min(128, max(32, -(-(-(-d.units * d.maxnb // (2 * sms))) // 32) * 32))
+        return {"sel": d.units * -(-d.maxnb // chunk), "spec": d.units * d.P,
+                "tasks": d.units * (1 + d.K + d.group)}
 
     def enable_trace(self, on: bool = True) -> None:
         """Record start/end times of every work item of the fused launches."""
@@ -122,28 +146,90 @@ class PRRDecoder:
         """Timeline of the last traced fused launch, per item kind (see summarize_trace)."""
         if self.trace is None:
             raise RuntimeError("tracing is off: call enable_trace() before the step")
-        return summarize_trace(self.trace.cpu().numpy(), self.fused_items())
+        return summarize_trace(self.trace.cpu().numpy())
+
+    STAT_NAMES = ("tie_mask_units", "key_search_units", "take_all_units", "spec_attended",
+                  "spec_skipped", "repaired", "reserved6", "reserved7")
+
+    def enable_stats(self, on: bool = True) -> None:
+        """Count, over the following steps, which finisher path each unit took and how
+        many speculative and repair blocks were attended or skipped (int64 [8] on the
+        device, added to by the kernels; read it with stats_dict)."""
+        self.stats = torch.zeros((8,), dtype=torch.int64, device=self.device) if on else None
+
+    def stats_dict(self) -> dict:
+        if self.stats is None:
+            raise RuntimeError("counters are off: call enable_stats() before the steps")
+        return dict(zip(self.STAT_NAMES, (int(x) for x in self.stats.cpu().tolist())))
+
 
     # ------------------------------------------------------------------ setup
-    def prefill(self, k: torch.Tensor, v: torch.Tensor, n0: int) -> None:
-        """Copy an initial context of n0 tokens ([B][Hkv][n0][d] bf16) into the cache,
-        build all block summaries, reset the EMA and predict from the zero state."""
+    def load_context(self, b: int, h: int, k: torch.Tensor, v: torch.Tensor) -> None:
+        """Write tokens [0, n) of sequence b, KV head h (k, v: [n][d] bf16 on the device)
+        into the cache, through the block table when the cache is paged."""
+        n, bs = k.shape[0], self.dims.bs
+        if self.block_table is None:
+            self.k_cache[b, h, :n].copy_(k)
+            self.v_cache[b, h, :n].copy_(v)
+            return
+        nbk = -(-n // bs)
+        pages = self.block_table[b, :nbk].long()
+        pad = nbk * bs - n  # rows past n in the last page are never read
+        kp = torch.nn.functional.pad(k, (0, 0, 0, pad)).view(nbk, bs, -1)
+        vp = torch.nn.functional.pad(v, (0, 0, 0, pad)).view(nbk, bs, -1)
+        self.k_cache[pages, h] = kp
+        self.v_cache[pages, h] = vp
+
+    def prefill(self, k: Optional[torch.Tensor], v: Optional[torch.Tensor], n0) -> None:
+        """Start decoding after an initial context: optionally copy it in (k, v
+        [B][Hkv][n0][d] bf16, contiguous caches only; else load_context wrote it), set the
+        sequence lengths (n0: one length, or one per sequence), build all block
+        summaries, reset the EMA and predict from the zero state."""
         d = self.dims
+        lens = [int(n0)] * d.B if isinstance(n0, int) else [int(x) for x in n0]
         with torch.cuda.stream(self.select_stream):
-            self.k_cache[:, :, :n0].copy_(k)
-            self.v_cache[:, :, :n0].copy_(v)
-            self.seq_lens.fill_(n0)
+            if k is not None:
+                self.k_cache[:, :, :lens[0]].copy_(k)
+                self.v_cache[:, :, :lens[0]].copy_(v)
+            self.seq_lens.copy_(torch.tensor(lens, dtype=torch.int32))
             self.ema.zero_()
             self.pred_buf.fill_(-1)
             _abi.prr_workspace_init(self.ws, self.select_stream)
             zeros = torch.zeros((d.B,), dtype=torch.int32, device=self.device)
-            ends = torch.full((d.B,), n0, dtype=torch.int32, device=self.device)
-            _abi.prr_update_summaries(d, self.k_cache, zeros, ends, None, n0, self.summ, self.ws,
+            ends = torch.tensor(lens, dtype=torch.int32, device=self.device)
+            _abi.prr_update_summaries(d, self.k_cache, zeros, ends, None, max(lens), self.summ, self.ws,
                                       self.select_stream)
             self.parity = 0
             if d.P > 0:
                 _abi.prr_ema_predict(d, self.ema, None, self.seq_lens, self.pred_buf[0], self.ws,
                                      self.select_stream)
+        self.select_stream.synchronize()
+
+    # ------------------------------------------------------------------ checkpoint / resume
+    def checkpoint(self) -> dict:
+        """Host copies of the state a decode step carries to the next one: the caches,
+        sequence lengths, block summaries, EMA state and the current prediction Pred_t
+        (and the block table of a paged cache).  The workspace holds nothing that
+        outlives a step, so it is not part of the state."""
+        self.select_stream.synchronize()
+        ck = {"k_cache": self.k_cache.cpu(), "v_cache": self.v_cache.cpu(), "seq_lens": self.seq_lens.cpu(),
+              "summ": self.summ.cpu(), "ema": self.ema.cpu(), "pred": self.pred.cpu()}
+        if self.block_table is not None:
+            ck["block_table"] = self.block_table.cpu()
+        return ck
+
+    def restore(self, ck: dict) -> None:
+        """Load a checkpoint() into this decoder (same dims): the next step continues
+        exactly where the checkpointed decoder stopped."""
+        with torch.cuda.stream(self.select_stream):
+            for name in ("k_cache", "v_cache", "seq_lens", "summ", "ema"):
+                getattr(self, name).copy_(ck[name])
+            if self.block_table is not None:
+                self.block_table.copy_(ck["block_table"])
+                self.table_host = ck["block_table"].numpy().copy()
+            self.parity, self.fused_parity = 0, 0
+            self.pred_buf[0].copy_(ck["pred"])
+            _abi.prr_workspace_init(self.ws, self.select_stream)
         self.select_stream.synchronize()
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
@@ -153,26 +239,32 @@ class PRRDecoder:
 
     # ------------------------------------------------------------------ the step
     def step(self, q: Optional[torch.Tensor] = None, timing: Optional[dict] = None,
-             swap: bool = True) -> None:
+             swap: bool = True, append: bool = False) -> None:
         """One decode step on the state's streams (q [B][Hq][d] bf16 is copied into the
         step's query buffer first when given).  Swaps Pred_t / Pred_{t+1} afterwards."""
         if q is not None:
             with torch.cuda.stream(self.select_stream):
                 self.q.copy_(q)
-        _abi.prr_decode_step(self.dims, self.buffers(), self.ws, self.select_stream,
+        _abi.prr_decode_step(self.dims, self.buffers(append=append), self.ws, self.select_stream,
                              self.spec_stream, self.events(timing))
         if swap and self.dims.P > 0:
             self.parity ^= 1
 
     def step_fused(self, q: Optional[torch.Tensor] = None, stream=None, swap: bool = True,
-                   parity: Optional[int] = None) -> None:
-        """The same step as one persistent launch on `stream` (default: select_stream)."""
+                   parity: Optional[int] = None, k_new: Optional[torch.Tensor] = None,
+                   v_new: Optional[torch.Tensor] = None, append: bool = False) -> None:
+        """The same step as one persistent launch on `stream` (default: select_stream).
+        With k_new / v_new ([B][Hkv][d] bf16, copied into the decoder's token buffers)
+        or `append`, the launch also appends the step's token (no separate append)."""
         st = stream or self.select_stream
-        if q is not None:
-            with torch.cuda.stream(st):
+        with torch.cuda.stream(st):
+            if q is not None:
                 self.q.copy_(q)
+            if k_new is not None:
+                self.k_new.copy_(k_new)
+                self.v_new.copy_(v_new)
         par = self.fused_parity if parity is None else parity
-        _abi.prr_decode_step_fused(self.dims, self.buffers(), self.ws, par, st)
+        _abi.prr_decode_step_fused(self.dims, self.buffers(append=append or k_new is not None), self.ws, par, st)
         if parity is None:
             self.fused_parity ^= 1
         if swap and self.dims.P > 0:
@@ -182,22 +274,28 @@ class PRRDecoder:
         return _abi.prr_get_device_status(self.ws)
 
 
-def summarize_trace(trace, items: dict) -> dict:
+KINDS = {1: "sel", 2: "spec", 3: "repair", 4: "ema", 5: "combine"}
+
+
+def summarize_trace(trace) -> dict:
     """Per item kind of one fused launch: how many items ran, when the first and last
     started and the last ended (microseconds after the earliest start), and the p50 /
-    mean / max item duration.  `trace` is the [items][4] record of prr_step_buffers
-    (start ns, end ns, SM << 32 | CTA, item), `items` the kind counts in queue order."""
+    mean / max item duration.  `trace` is the [records][4] array of prr_step_buffers
+    (start ns, end ns, SM << 32 | group << 16 | CTA, kind | finisher ns << 32)."""
     import numpy as np
     tr = np.asarray(trace, dtype=np.int64)
     ran = tr[:, 0] > 0
     if not ran.any():
         return {}
     t0 = tr[ran, 0].min()
-    out, off = {}, 0
-    for kind, cnt in items.items():
-        seg = tr[off:off + cnt]
-        off += cnt
-        seg = seg[seg[:, 0] > 0]
+    out = {"end_us": float((tr[ran, 1].max() - t0) / 1e3)}
+    kinds = tr[:, 3] & 0xFFFFFFFF
+    fin = (tr[:, 3] >> 32) / 1e3
+    if (fin > 0).any():
+        f = fin[fin > 0]
+        out["finisher"] = {"n": int(len(f)), "dur_p50_us": float(np.median(f)), "dur_max_us": float(f.max())}
+    for code, kind in KINDS.items():
+        seg = tr[ran & (kinds == code)]
         if len(seg) == 0:
             out[kind] = {"n": 0}
             continue

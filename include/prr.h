@@ -15,10 +15,11 @@
  *    allocates, frees or synchronises device memory; only prr_get_device_status
  *    synchronises (to read the status word back).
  *  - bf16 arrays are passed as uint16_t bit patterns.
- *  - Shapes (row-major, innermost last), with units = B*Hkv, G = Hq/Hkv,
- *    maxnb = ceil(cap_tokens/bs):
+ *  - Shapes (row-major, innermost last), with units = B*Hkv (B*Hq under
+ *    PRR_SELECT_PER_HEAD), G = Hq/Hkv, maxnb = ceil(cap_tokens/bs):
  *      q            [B][Hq][d]               bf16   query of the step
- *      k_cache/v_cache [B][Hkv][cap_tokens][d] bf16 (16-byte aligned base)
+ *      k_cache/v_cache [B][Hkv][cap_tokens][d] bf16 (16-byte aligned base), or a paged
+ *                   pool [pages][Hkv][bs][d] with a block table (see prr_dims)
  *      seq_lens     [B]                      int32  tokens n in the cache, 1 <= n <= cap
  *      summ         [B][Hkv][maxnb][2][d]    bf16   per block: min row then max row
  *      ema          [B][Hkv][maxnb]          fp64   EMA state, starts at 0
@@ -71,7 +72,7 @@ typedef enum {
 #define PRR_DEV_BAD_PRED 2     /* predicted list entry out of range or not ascending */
 #define PRR_DEV_BAD_MISSED 3   /* missed list entry out of range */
 #define PRR_DEV_WAIT_TIMEOUT 4 /* a bounded wait for a TMA copy gave up */
-#define PRR_DEV_BAD_RANGE 5    /* summary update range outside [0, cap_tokens] */
+#define PRR_DEV_BAD_RANGE 5    /* summary update range outside [0, cap_tokens], or a block-table entry outside [0, pages) */
 
 typedef struct {
   int32_t B;          /* sequences */
@@ -84,7 +85,37 @@ typedef struct {
   int32_t P;          /* speculation budget: predicted blocks per (sequence, KV head) */
   double alpha;       /* EMA decay, 0 <= alpha <= 1 */
   float scale;        /* softmax scale applied to q.k (usually 1/sqrt(d)) */
+  /* Block selector (the DSA method whose top-K PRR accelerates; PRR abstract: results
+   * across representative DSA methods).  Zero-initialised dims give the default.
+   *   PRR_SELECT_GROUP_SUM  one selection per KV head; block score = the sum over the
+   *                         group's query heads of each head's Quest bound
+   *   PRR_SELECT_GROUP_MAX  one selection per KV head; score = the largest of the
+   *                         group's per-head bounds
+   *   PRR_SELECT_PER_HEAD   every query head selects its own top-K with its own bound;
+   *                         then a "unit" is a (sequence, query head) pair, and the
+   *                         per-unit arrays below are [B][Hq][...] instead of
+   *                         [B][Hkv][...] (summaries and KV stay per KV head). */
+  int32_t selector;
+  int32_t n_sink;     /* the first n_sink blocks are always selected (attention sinks), 0..2^22 */
+  int32_t n_local;    /* the newest n_local blocks are always selected (local window), 0..2^22;
+                       * the rest of the min(K, nb) budget goes to the best other blocks; when
+                       * the forced blocks alone exceed it, sinks come first (lowest index
+                       * first), then local blocks from the newest backwards */
+  /* KV cache layout.  pages == 0 (block_table NULL): contiguous, k_cache / v_cache
+   * [B][Hkv][cap_tokens][d].  pages > 0: paged (as in PagedAttention / vLLM and
+   * FlashInfer serving, in PRR's reference list) -- k_cache / v_cache are pools of
+   * `pages` pages [pages][Hkv][bs][d], one page holding one block of bs tokens of every
+   * KV head, and block_table (device int32 [B][maxnb]) maps block j of sequence b to its
+   * page.  cap_tokens stays the per-sequence capacity.  Only entries of blocks below a
+   * sequence's length are read; an entry outside [0, pages) sets PRR_DEV_BAD_RANGE and
+   * that block is not read. */
+  int32_t pages;
+  const int32_t* block_table;
 } prr_dims;
+
+#define PRR_SELECT_GROUP_SUM 0
+#define PRR_SELECT_GROUP_MAX 1
+#define PRR_SELECT_PER_HEAD 2
 
 /* Buffers of one decode step (see the shapes above). */
 typedef struct {
@@ -105,13 +136,31 @@ typedef struct {
   float* part_O;
   float* out;
   float* lse;
-  /* Optional (NULL: off).  prr_decode_step_fused records, for every work item i of the
-   * launch, trace[4i..4i+3] = {start ns, end ns, (SM id << 32) | CTA, i} (%globaltimer).
-   * Items, in order: units*ceil(maxnb/C) selection chunks (C = ceil(units*maxnb/512)
-   * rounded up to a multiple of 32, clamped to [32, 128]), units finishers,
-   * units predictor updates, units*P speculative slots, units*R repair items
-   * (R = min(K, max(4, ceil(1024/units)))), units*G merges. */
+  /* Optional, both or neither (NULL: the caller appended the step's token already).
+   * The step's new token [B][Hkv][d] bf16 (16-byte aligned).  The step then appends it
+   * itself: it writes the rows at position seq_lens[b] of the caches, works on
+   * seq_lens[b] + 1 tokens and advances seq_lens[b] when it is done (a full cache sets
+   * PRR_DEV_BAD_SEQ_LEN and skips that sequence).  prr_decode_step_fused does this
+   * inside its one launch; prr_decode_step launches the append first. */
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  /* Optional (NULL: off).  prr_decode_step_fused records, for every item its CTAs run,
+   * trace[4i..4i+3] = {start ns, end ns, (SM id << 32) | (consumer group << 16) | CTA,
+   * kind | (finisher ns << 32)} (%globaltimer; kind 1 selection chunk, 2 speculative
+   * block, 3 repair block, 4 predictor update, 5 merge; a selection chunk that ran its
+   * unit's top-K records the top-K's duration in the high half).  Records: first the main work in queue order --
+   * units*ceil(maxnb/C) selection chunks (C blocks each: units*maxnb/(2*SMs) rounded up
+   * to a multiple of 32, clamped to [32, 128]), then units*P speculative slots -- then
+   * units*(1+K+G) task records in the order the tasks were queued.  Items that did not
+   * run stay zero.  Size: 4 * (units*(ceil(maxnb/C) + P) + units*(1+K+G)) words. */
   unsigned long long* trace;
+  /* Optional (NULL: off).  Eight counters the step adds to (atomically; the caller
+   * zeroes them):  [0] units whose top-K came straight from the 32-block group tie
+   * masks, [1] units whose top-K needed the search over the block keys, [2] units
+   * that took every block (K_eff = nb), [3] speculative blocks attended, [4]
+   * speculative blocks skipped because selection had already dropped them, [5]
+   * repaired (missed) blocks attended, [6], [7] zero. */
+  unsigned long long* stats;
 } prr_step_buffers;
 
 /* Events of one decode step.  fork, sel_done, spec_done and join are required (any
@@ -145,6 +194,14 @@ const char* prr_status_string(prr_status s);
  * 32-bit score key per block, one (max key, tie mask) summary per 32-block group, the
  * repair partials and the fused step's control words (two copies, one per parity). */
 size_t prr_workspace_bytes(const prr_dims* dims);
+
+/* Byte offset of a workspace word reserved for failure-detection tests.  A test may set
+ * it to a non-zero int32 (with a plain copy into the workspace) to make
+ * prr_decode_step_fused skip its selection chunks: no unit's top-K completes, so the
+ * launch's end-of-step wait runs out after its one-second limit and the launch returns
+ * with the device status PRR_DEV_WAIT_TIMEOUT, without a fault.  Leave it zero
+ * otherwise; prr_workspace_init clears it. */
+#define PRR_WS_TEST_SKIP_SELECTION_OFFSET 4
 
 /* Zero-fill a workspace (required once before first use, and after a device error).
  * The kernels leave their tickets re-armed, so steady-state calls need no reset. */
@@ -232,14 +289,20 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* buf, vo
                            size_t ws_bytes, cudaStream_t select_stream, cudaStream_t spec_stream,
                            const prr_step_events* events);
 
-/* The same decode step (a1-a7) in ONE persistent launch on `stream`.  Resident CTAs
- * take work from a queue ordered selection -> speculation -> repair -> predictor ->
- * merge; speculation overlaps selection inside the launch, a speculative block that
- * selection has already dropped is skipped, and dependent work waits (bounded) only on
- * earlier queue entries.  step_parity (0 or 1) must alternate between consecutive
- * calls that share `ws`: each launch uses one copy of the workspace control words and
- * clears the other for the next launch.  Same buffers, results and error behaviour as
- * prr_decode_step; capturable in a CUDA graph (one graph per parity).
+/* The same decode step (a1-a7) in ONE persistent launch on `stream`: one CTA per SM, a
+ * producer warp that keeps the K/V and summary copies of the next items in flight and
+ * two consumer groups that compute.  Selection chunks are handed out first, then
+ * speculation; the consumer that scores a unit's last chunk runs its top-K at once
+ * and queues the unit's repairs and predictor update, and the unit's last partial
+ * queues its merges, so no work item waits for another.  A speculative block that
+ * selection has already dropped is skipped.  step_parity (0 or 1) must alternate
+ * between consecutive calls that share `ws`: each launch uses one copy of the
+ * workspace control words and clears the other for the next launch.  Same buffers,
+ * results and error behaviour as prr_decode_step; capturable in a CUDA graph (one
+ * graph per parity).  Size limit: each shared-memory slot must hold the finisher's
+ * and the predictor's per-unit scratch, about 12*maxnb bytes, next to two K/V tiles;
+ * dims whose slots no longer fit twice in 227 KB (maxnb beyond roughly 12,000 blocks)
+ * return PRR_ERR_SHAPE -- prr_decode_step has no such limit below 50,000 blocks.
  * PRR abstract / method summary: speculation overlaps selection and stays off the
  * critical path; repair merges the missed blocks without recomputation. */
 prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* buf, void* ws,
@@ -265,7 +328,7 @@ prr_status prr_budget_fit(const double* context_tokens, const double* us, int32_
 prr_status prr_budget_choose(const double* sel_coef, const double* spec_coef, const int32_t* p_grid,
                              int32_t np, int32_t degree, int32_t context_tokens, int32_t* p_out);
 
-/* Largest B*Hkv*ceil(cap_tokens/bs) that prr_select_topk_static accepts, and the bytes
+/* Largest units*ceil(cap_tokens/bs) that prr_select_topk_static accepts, and the bytes
  * of device memory its fixed scratch array occupies on every GPU that loads the
  * library (status word + 65536 chunk tickets + one 32-bit key per block). */
 #define PRR_SELECT_STATIC_MAX_BLOCKS (1 << 20)
@@ -286,7 +349,7 @@ prr_status prr_budget_choose(const double* sel_coef, const double* spec_coef, co
  *   status: optional device int32; receives this call's device-side status code
  *           (0 = ok, else one of PRR_DEV_*), written on `stream` after the kernel.
  * Returns PRR_ERR_CAPACITY, without enqueuing anything, when
- * B*Hkv*ceil(cap_tokens/bs) > PRR_SELECT_STATIC_MAX_BLOCKS.  Calls no cudaMalloc,
+ * units*ceil(cap_tokens/bs) > PRR_SELECT_STATIC_MAX_BLOCKS.  Calls no cudaMalloc,
  * cudaFree or other allocating routine.  The first call in each CUDA context (made
  * with that context current) looks up the array's device address and keeps it for
  * that context, so a context created later on the same device (for instance after

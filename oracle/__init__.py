@@ -66,6 +66,8 @@ class Oracle:
         L.oracle_top_ranked.argtypes = [_f64p, _int, _int, _i32p]
         L.oracle_block_scores_max.argtypes = [_f64p, _int, _int, _f64p, _f64p, _int, _f64p]
         L.oracle_top_ranked_forced.argtypes = [_f64p, _int, _int, _int, _int, _i32p]
+        L.oracle_gather_pages.argtypes = [_u16p, _i32p, _int, _int, _int, _int, _int, _u16p]
+        L.oracle_block_scores_rep.argtypes = [_f64p, _int, _int, _u16p, _int, _int, _i32p, _int, _int, _f64p]
         L.oracle_top_ranked_forced.restype = _int
         L.oracle_top_ranked.restype = _int
         L.oracle_ema_update.argtypes = [_f64p, _int, _i32p, _int, _dbl]
@@ -133,6 +135,27 @@ class Oracle:
         out = np.zeros(max(min(K, len(v)), 1), np.int32)
         cnt = self.L.oracle_top_ranked_forced(v, len(v), K, n_sink, n_local, out)
         return out[:cnt]
+
+    def block_scores_rep(self, q, k_bits, n, bs, rep):
+        """Selector variant (InfLLM-style): each block scored by r representative tokens
+        of its own (rep [nb][r] offsets in the block), summed over heads and tokens."""
+        q = _c(q, np.float64)
+        G, d = q.shape
+        rep = _c(rep, np.int32)
+        nb, r = rep.shape
+        out = np.zeros(nb, np.float64)
+        self.L.oracle_block_scores_rep(q, G, d, _c(k_bits, np.uint16), n, bs, rep, r, nb, out)
+        return out
+
+    def gather_pages(self, pool_bits, table_row, h, n, bs):
+        """Tokens [0, n) of KV head h of one sequence from a paged pool
+        [pages][Hkv][bs][d] through the sequence's block-table row, as [n][d] bits."""
+        pool_bits = _c(pool_bits, np.uint16)
+        _, Hkv, bs_, d = pool_bits.shape
+        assert bs_ == bs
+        out = np.zeros((n, d), np.uint16)
+        self.L.oracle_gather_pages(pool_bits, _c(table_row, np.int32), Hkv, h, n, bs, d, out)
+        return out
 
     def select_per_head(self, q, smin, smax, K):
         """Selector variant: every query head selects with its own bound (no sharing)."""

@@ -213,6 +213,50 @@ int oracle_top_ranked_forced(const double *v, int nb, int K, int n_sink, int n_l
     return keff;
 }
 
+/* InfLLM-style representative-key scores (InfLLM: Training-Free Long-Context
+ * Extrapolation for LLMs with an Efficient Context Memory, in PRR's reference list;
+ * only its title is on the pages).  Each block is represented by r of its own tokens
+ * instead of a min/max summary; which tokens is decided when the block is built (an
+ * input here, rep [nb][r] offsets inside the block).  The block score is the sum over
+ * the group's query heads and the representatives of q_h . k_rep:
+ *   s_b = sum_h sum_j q_h . k[b*bs + min(rep[b][j], valid_b - 1)],
+ * valid_b = the block's tokens below n (a representative past a ragged tail stands
+ * for the block's last token).  q is [G][d] (widened), k one slice [tokens][d] bits. */
+void oracle_block_scores_rep(const double *q, int G, int d, const uint16_t *k, int n, int bs,
+                             const int32_t *rep, int r, int nb, double *s)
+{
+    for (int b = 0; b < nb; ++b) {
+        int valid = n - b * bs;
+        if (valid > bs) valid = bs;
+        double total = 0.0;
+        for (int h = 0; h < G; ++h) {
+            for (int j = 0; j < r; ++j) {
+                int off = rep[(size_t)b * r + j];
+                if (off > valid - 1) off = valid - 1;
+                if (off < 0) off = 0;
+                const uint16_t *krow = k + ((size_t)b * bs + off) * d;
+                for (int c = 0; c < d; ++c) total += q[h * d + c] * bf16_val(krow[c]);
+            }
+        }
+        s[b] = total;
+    }
+}
+
+/* Paged KV cache (the PagedAttention / vLLM and FlashInfer layouts in PRR's reference
+ * list; only their titles are on the pages): a pool of pages [pages][Hkv][bs][d], one
+ * page holding one block of bs tokens of every KV head, and per sequence a block table
+ * giving the page of each block.  This gathers tokens [0, n) of KV head h of one
+ * sequence (table = that sequence's row) into a contiguous [n][d] slice, on which every
+ * function above applies unchanged. */
+void oracle_gather_pages(const uint16_t *pool, const int32_t *table, int Hkv, int h, int n, int bs, int d,
+                         uint16_t *out)
+{
+    for (int t = 0; t < n; ++t) {
+        const uint16_t *src = pool + (((size_t)table[t / bs] * Hkv + h) * bs + t % bs) * d;
+        memcpy(out + (size_t)t * d, src, sizeof(uint16_t) * d);
+    }
+}
+
 /* ------------------------------------------------------------------ 5. EMA */
 
 /* e_b <- alpha*e_b + beta*[b in S] for every b < nb, beta = 1 - alpha. */

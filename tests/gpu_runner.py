@@ -2,6 +2,7 @@
 and through the fp64 oracle, step by step, and collect a comparison report."""
 from __future__ import annotations
 
+import dataclasses
 from typing import Dict, Iterable, List, Optional, Sequence, Tuple
 
 import numpy as np
@@ -19,19 +20,30 @@ def to_dev_bits(a: np.ndarray, device="cuda") -> torch.Tensor:
     return t.to(device).view(torch.bfloat16)
 
 
-def make_decoder(w: W.Workload, steps: int, cap_extra: int = 0) -> Tuple[PRRDecoder, Dims]:
+def shuffled_block_table(w: W.Workload, maxnb: int, spare: int, seed: int = 5):
+    """A paged layout for the test: every block of every sequence gets its own page, the
+    pages in a seeded random order inside a pool with `spare` pages left unused."""
+    pages = w.B * maxnb + spare
+    perm = np.random.default_rng(seed).permutation(pages)[:w.B * maxnb]
+    return torch.from_numpy(perm.astype(np.int32).reshape(w.B, maxnb)), pages
+
+
+def make_decoder(w: W.Workload, steps: int, cap_extra: int = 0, paged: bool = False) -> Tuple[PRRDecoder, Dims]:
     cap = w.N0 + steps + cap_extra
     dims = Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, bs=w.bs, cap_tokens=cap, K=w.K, P=w.P,
-                alpha=w.alpha)
-    dec = PRRDecoder(dims)
+                alpha=w.alpha, selector=w.selector, n_sink=w.n_sink, n_local=w.n_local)
+    table = None
+    if paged:
+        table, pages = shuffled_block_table(w, dims.maxnb, spare=7)
+        dims = dataclasses.replace(dims, pages=pages)
+    dec = PRRDecoder(dims, block_table=table)
     for b in range(w.B):
         for h in range(w.Hkv):
-            k0, v0 = W.kv_prefix(w, b, h)
-            dec.k_cache[b, h, :w.N0].copy_(to_dev_bits(k0))
-            dec.v_cache[b, h, :w.N0].copy_(to_dev_bits(v0))
+            k0, v0 = W.kv_prefix(w, b, h, w.n0(b))
+            dec.load_context(b, h, to_dev_bits(k0), to_dev_bits(v0))
     torch.cuda.synchronize()
-    dec.prefill(dec.k_cache[:, :, :w.N0], dec.v_cache[:, :, :w.N0], w.N0)
-    return dec, dims
+    dec.prefill(None, None, [w.n0(b) for b in range(w.B)])
+    return dec, dec.dims
 
 
 def appended_tokens(w: W.Workload, steps: int):
@@ -46,30 +58,39 @@ def appended_tokens(w: W.Workload, steps: int):
 
 def run_parity(w: W.Workload, steps: int, units: Optional[Sequence[Tuple[int, int]]] = None,
                forced: Optional[Tuple[float, int]] = None, graph: bool = False,
-               mode: str = "fused") -> Report:
+               mode: str = "fused", append: str = "host", paged: bool = False) -> Report:
     """Compare `steps` decode steps.  `units` samples the (b, kvh) pairs the oracle
     follows (default: all).  `forced` = (overlap, level) replaces the predictor's output
     with a predicted set forced to that overlap with the oracle's true set (all units
     are then followed).  `mode` selects the step implementation: "fused" (one
-    persistent launch) or "streams" (two streams, one launch per kernel)."""
+    persistent launch) or "streams" (two streams, one launch per kernel).  `append`
+    selects who appends each step's token: "host" (prr_append_kv before the step) or
+    "step" (the step itself, from the decoder's k_new / v_new buffers).  `paged` puts
+    the KV cache in a pool of pages in shuffled order behind a block table."""
     o = OR.default()
-    all_units = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    all_units = [(b, h) for b in range(w.B) for h in range(w.sel_heads)]
     if units is None or forced is not None:
         units = all_units
     uo: Dict[Tuple[int, int], UnitOracle] = {u: UnitOracle.create(w, u[0], u[1], steps, o) for u in units}
-    dec, dims = make_decoder(w, steps)
+    dec, dims = make_decoder(w, steps, paged=paged)
     kn, vn = appended_tokens(w, steps)
     qs = W.queries(w, steps)
     rep = Report()
     gaussian = w.qk == "gauss"
     graphs = {}
+    in_step = append == "step"
     for t in range(steps):
-        dec.append(to_dev_bits(kn[t]), to_dev_bits(vn[t]))
+        if in_step:  # on the step's stream, ahead of the launch that reads them
+            with torch.cuda.stream(dec.select_stream):
+                dec.k_new.copy_(to_dev_bits(kn[t]))
+                dec.v_new.copy_(to_dev_bits(vn[t]))
+        else:
+            dec.append(to_dev_bits(kn[t]), to_dev_bits(vn[t]))
         q_dev = to_dev_bits(qs[t])
         sel_info = {u: uo[u].select(t, qs[t]) for u in units}
         if forced is not None:
             overlap, level = forced
-            pred_host = np.full((w.B, w.Hkv, w.P), -1, np.int32)
+            pred_host = np.full((w.B, w.sel_heads, w.P), -1, np.int32)
             for (b, h), (n, nb, qg, s, sel) in sel_info.items():
                 fp = W.forced_prediction(w, sel, nb, overlap, level, t, b, h)
                 pred_host[b, h, :len(fp)] = fp
@@ -82,9 +103,9 @@ def run_parity(w: W.Workload, steps: int, units: Optional[Sequence[Tuple[int, in
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=dec.select_stream):
                     if mode == "fused":
-                        dec.step_fused(swap=False, parity=dec.fused_parity)
+                        dec.step_fused(swap=False, parity=dec.fused_parity, append=in_step)
                     else:
-                        dec.step(swap=False)
+                        dec.step(swap=False, append=in_step)
                 graphs[key] = g
             dec.q.copy_(q_dev)
             torch.cuda.synchronize()
@@ -94,9 +115,9 @@ def run_parity(w: W.Workload, steps: int, units: Optional[Sequence[Tuple[int, in
             if dims.P > 0:
                 dec.parity ^= 1
         elif mode == "fused":
-            dec.step_fused(q_dev)
+            dec.step_fused(q_dev, append=in_step)
         else:
-            dec.step(q_dev)
+            dec.step(q_dev, append=in_step)
         torch.cuda.synchronize()
         status = dec.device_status()
         if status != 0:
@@ -129,7 +150,7 @@ def run_parity(w: W.Workload, steps: int, units: Optional[Sequence[Tuple[int, in
             keep_ref[:len(res["keep"])] = res["keep"]
             if w.P > 0 and not np.array_equal(g_keep[b, h], keep_ref):
                 rep.fail(f"{tag}: keep differs gpu={g_keep[b, h].tolist()} oracle={keep_ref.tolist()}")
-            rows = slice(h * w.G, (h + 1) * w.G)
+            rows = u.qrows
             compare_attention(rep, tag, g_out[b, rows], g_lse[b, rows], res["out"], res["lse"])
             if not np.array_equal(g_ema[b, h, :nb], u.ema[:nb]):
                 bad = np.nonzero(g_ema[b, h, :nb] != u.ema[:nb])[0][:5]
@@ -141,4 +162,8 @@ def run_parity(w: W.Workload, steps: int, units: Optional[Sequence[Tuple[int, in
         if rep.messages:
             return rep
     rep.check_near_ties()
+    got_lens = dec.seq_lens.cpu().numpy()
+    want = [w.n0(b) + steps for b in range(w.B)]
+    if got_lens.tolist() != want:
+        rep.fail(f"seq_lens after {steps} steps: {got_lens.tolist()}, expected {want}")
     return rep

@@ -399,9 +399,66 @@ def check_selector_variants(o):
         assert np.array_equal(o.top_ranked_forced(v, K, 0, 0), o.top_ranked(v, K))
 
 
+def check_rep_scores(o):
+    """Representative-key scores: with every token of full blocks as a representative
+    they equal the sum of the group's queries dotted with the block's key sum (numpy);
+    with one token per block they are r times that token's dot product; a
+    representative past a ragged tail stands for the block's last valid token; top-K
+    over them matches brute-force enumeration."""
+    rng = np.random.default_rng(41)
+    G, d, bs = 3, 16, 8
+    n = 8 * bs
+    q = _f(_grid_bits(rng, (G, d)))
+    k = _grid_bits(rng, (n, d))
+    kf = _f(k)
+    rep = np.tile(np.arange(bs, dtype=np.int32), (n // bs, 1))
+    s = o.block_scores_rep(q, k, n, bs, rep)
+    ref = np.array([q.sum(0) @ kf[b * bs:(b + 1) * bs].sum(0) for b in range(n // bs)])
+    assert np.allclose(s, ref, rtol=0, atol=1e-12)
+    r = 3
+    s1 = o.block_scores_rep(q, k, n, 1, np.zeros((n, r), np.int32))
+    assert np.allclose(s1, r * (kf @ q.sum(0)), rtol=0, atol=1e-12)
+    # ragged tail: n = 5*bs + 3, block 5 holds 3 tokens; offsets 6 and 7 mean token 2
+    n2 = 5 * bs + 3
+    rep2 = np.array([[0, 6], [1, 7], [2, 2], [3, 0], [4, 5], [1, 7]], np.int32)
+    s2 = o.block_scores_rep(q, k[:n2], n2, bs, rep2)
+    qs = q.sum(0)
+    assert abs(s2[5] - qs @ (kf[5 * bs + 1] + kf[5 * bs + 2])) < 1e-12
+    assert abs(s2[1] - qs @ (kf[bs + 1] + kf[bs + 7])) < 1e-12
+    for trial in range(20):
+        nbt = int(rng.integers(1, 9))
+        rep3 = rng.integers(0, bs, size=(nbt, 2)).astype(np.int32)
+        v = o.block_scores_rep(q, k[:nbt * bs], nbt * bs, bs, rep3)
+        K = int(rng.integers(1, 4))
+        assert list(o.top_ranked(v, K)) == _brute_topk(v, K)
+
+
+def check_paged_gather(o):
+    """Gathering a sequence through its block table from a pool whose pages hold the
+    blocks in a shuffled order gives back the contiguous slice (numpy scatter), so
+    summaries, scores and attention on the gathered slice are the contiguous ones."""
+    rng = np.random.default_rng(43)
+    Hkv, bs, d = 3, 8, 16
+    for n in (5 * bs, 5 * bs - 3, 1):
+        nbk = -(-n // bs)
+        pages = nbk * 2 + 3
+        k = _grid_bits(rng, (Hkv, nbk * bs, d))
+        table = rng.permutation(pages)[:nbk].astype(np.int32)
+        pool = np.zeros((pages, Hkv, bs, d), np.uint16)
+        for j in range(nbk):
+            pool[table[j]] = k[:, j * bs:(j + 1) * bs]
+        for h in range(Hkv):
+            g = o.gather_pages(pool, table, h, n, bs)
+            assert np.array_equal(g, k[h, :n]), (n, h)
+            lo, hi = o.build_summaries(g, n, bs)
+            lo2, hi2 = o.build_summaries(k[h, :n], n, bs)
+            assert np.array_equal(lo, lo2) and np.array_equal(hi, hi2)
+
+
 ALL_CHECKS = [
     check_summaries_vs_numpy, check_bound_dominates_and_is_tight, check_grid_scores_exact,
     check_topk_bruteforce, check_ema_closed_form, check_ema_rounding_fixed, check_predict_from_zero_state,
     check_attention_vs_sdpa, check_prr_invariance, check_merge_of_two_token_sets,
-    check_hand_examples, check_decode_step_driver, check_selector_variants,
+    check_hand_examples, check_decode_step_driver, check_selector_variants, check_rep_scores,
+    check_paged_gather,
 ]

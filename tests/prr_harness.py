@@ -38,10 +38,12 @@ def f64(bits):
 
 @dataclass
 class UnitOracle:
-    """Oracle trajectory of one (sequence, KV head), driven step by step."""
+    """Oracle trajectory of one selection unit, driven step by step: a (sequence, KV
+    head) pair scored with the group's query heads, or, under per-head selection, a
+    (sequence, query head) pair scored with that head alone over its KV head's keys."""
     w: W.Workload
     b: int
-    kvh: int
+    kvh: int           # selection head: a KV head, or a query head under per-head selection
     k: np.ndarray      # [N0+steps][d] bits
     v: np.ndarray
     smin: np.ndarray
@@ -50,32 +52,50 @@ class UnitOracle:
     pred: np.ndarray   # Pred_t (ascending)
     o: OR.Oracle
 
+    @property
+    def kv_head(self) -> int:
+        return self.kvh // self.w.G if self.w.selector == "per_head" else self.kvh
+
+    @property
+    def qrows(self) -> slice:
+        if self.w.selector == "per_head":
+            return slice(self.kvh, self.kvh + 1)
+        return slice(self.kvh * self.w.G, (self.kvh + 1) * self.w.G)
+
     @classmethod
     def create(cls, w: W.Workload, b: int, kvh: int, steps: int, o: OR.Oracle):
-        k0, v0 = W.kv_prefix(w, b, kvh)
-        kn, vn = W.kv_appended(w, b, kvh, steps)
+        kv = kvh // w.G if w.selector == "per_head" else kvh
+        n0 = w.n0(b)
+        k0, v0 = W.kv_prefix(w, b, kv, n0)
+        kn, vn = W.kv_appended(w, b, kv, steps)
         k = np.concatenate([k0, kn])
         v = np.concatenate([v0, vn])
         maxnb = w.nb(w.N0 + steps)
         smin = np.zeros((maxnb, w.d))
         smax = np.zeros((maxnb, w.d))
-        lo, hi = o.build_summaries(k, w.N0, w.bs)
+        lo, hi = o.build_summaries(k, n0, w.bs)
         smin[:lo.shape[0]], smax[:lo.shape[0]] = lo, hi
         ema = np.zeros(maxnb)
-        pred = o.top_ranked(np.zeros(w.nb(w.N0)), w.P) if w.P > 0 else np.zeros(0, np.int32)
+        pred = o.top_ranked(np.zeros(w.nb(n0)), w.P) if w.P > 0 else np.zeros(0, np.int32)
         return cls(w, b, kvh, k, v, smin, smax, ema, pred, o)
 
     def select(self, t: int, q_bits: np.ndarray):
         """Summary update for token N0+t, scores, true top-K (all from the oracle)."""
         w, o = self.w, self.o
-        n = w.N0 + t + 1
+        n = w.n0(self.b) + t + 1
         nb = w.nb(n)
         tail = (n - 1) // w.bs
         lo, hi = o.block_summary(self.k, n, w.bs, tail)
         self.smin[tail], self.smax[tail] = lo, hi
-        qg = f64(q_bits[self.b, self.kvh * w.G:(self.kvh + 1) * w.G])
-        s = o.block_scores(qg, self.smin[:nb], self.smax[:nb])
-        sel = o.top_ranked(s, w.K)
+        qg = f64(q_bits[self.b, self.qrows])
+        if w.selector == "group_max":
+            s = o.block_scores_max(qg, self.smin[:nb], self.smax[:nb])
+        else:  # group sum, or one head's own bound under per-head selection
+            s = o.block_scores(qg, self.smin[:nb], self.smax[:nb])
+        if w.n_sink or w.n_local:
+            sel = o.top_ranked_forced(s, w.K, w.n_sink, w.n_local)
+        else:
+            sel = o.top_ranked(s, w.K)
         return n, nb, qg, s, sel
 
     def finish(self, n, nb, qg, sel, pred):
@@ -83,7 +103,7 @@ class UnitOracle:
         w, o = self.w, self.o
         missed, keep = o.missed_keep(sel, pred)
         outs, lses = [], []
-        for g in range(w.G):
+        for g in range(qg.shape[0]):
             out, lse = o.attend_blocks(qg[g], self.k, self.v, n, w.bs, sel, w.scale())
             outs.append(out)
             lses.append(lse)

@@ -292,6 +292,18 @@ def test_decode_ragged_small(mode):
 
 
 @pytest.mark.parametrize("mode", MODES)
+def test_decode_append_in_step(mode):
+    """The step appends its own token (k_new / v_new in the step buffers): the fused
+    launch writes the row, attends it from k_new / v_new and advances seq_lens itself;
+    the two-stream step launches the append first.  Same results as appending first."""
+    w = W.workload("tiny").with_(name="append_in_step", B=3, Hq=12, Hkv=3, d=128, N0=2000, bs=64, K=16,
+                                 P=16, steps=12, walk_p=0.8)
+    _assert_ok(run_parity(w, steps=12, mode=mode, append="step"))
+    w2 = w.with_(N0=1983, bs=128, K=8, P=8, steps=8)  # blocks of 128, new token mid-block
+    _assert_ok(run_parity(w2, steps=8, graph=True, mode=mode, append="step"))
+
+
+@pytest.mark.parametrize("mode", MODES)
 def test_decode_no_speculation(mode):
     """Budget P = 0: every selected block is repaired; the predictor is idle."""
     w = W.workload("tiny").with_(name="no_spec", B=2, Hq=8, Hkv=2, d=128, N0=3000, bs=64, K=16,
@@ -340,6 +352,127 @@ def test_decode_repair_sweep_full_size():
         _assert_ok(run_parity(w, steps=2, forced=(w.forced_overlaps[level], level)))
 
 
+def test_decode_full_size_append_in_step():
+    """The headline 128K batched workload with the token appended inside the fused
+    launch (the bench's end-to-end path), graphs, sampled units."""
+    _assert_ok(run_parity(W.workload("batched_128k"), steps=4, units=[(0, 0), (9, 2), (15, 7)], graph=True,
+                          append="step"))
+
+
+# ----------------------------------------------------------------------------- selector variants
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("selector,n_sink,n_local", [
+    ("group_max", 0, 0), ("per_head", 0, 0), ("group_sum", 2, 3), ("group_max", 1, 4), ("per_head", 1, 2),
+])
+def test_decode_selector_variants(mode, selector, n_sink, n_local):
+    """The selector variants of the representative DSA methods (group max of the
+    per-head bounds, per-query-head selection, forced sink and local blocks) through
+    both step implementations, every unit, against the oracle's variants."""
+    w = W.workload("tiny").with_(name="variant", B=2, Hq=8, Hkv=2, d=128, N0=3000, bs=64, K=12, P=12, steps=6,
+                                 walk_p=0.8, selector=selector, n_sink=n_sink, n_local=n_local)
+    _assert_ok(run_parity(w, steps=6, mode=mode))
+
+
+@pytest.mark.parametrize("selector", ["group_max", "per_head"])
+def test_decode_selector_variants_gqa8(selector):
+    """8:1 GQA at the 512K workload's head shape (reduced context), forced blocks, the
+    token appended inside the fused launch, CUDA graphs."""
+    w = W.workload("long_512k").with_(B=1, N0=60000, steps=4, selector=selector, n_sink=1, n_local=2)
+    _assert_ok(run_parity(w, steps=4, graph=True, append="step"))
+
+
+@pytest.mark.parametrize("selector,K,n_sink,n_local", [
+    ("group_max", 64, 0, 0), ("per_head", 16, 0, 0), ("group_sum", 3, 2, 4), ("group_sum", 20, 5, 5),
+    ("per_head", 8, 1, 1),
+])
+def test_select_topk_variants(selector, K, n_sink, n_local):
+    """prr_select_topk under each selector, bit-exact on the grid; (K=3, 2 sinks, 4
+    local) overflows the budget: sinks first, then the newest local block."""
+    rng = np.random.default_rng(31)
+    B, Hkv, G, d, bs, n = 2, 2, 4, 128, 64, 9000
+    dims = prr.Dims(B=B, Hq=G * Hkv, Hkv=Hkv, d=d, bs=bs, cap_tokens=n + 3, K=K, P=K, selector=selector,
+                    n_sink=n_sink, n_local=n_local)
+    k = _rng_grid(rng, (B, Hkv, n + 3, d))
+    q = _rng_grid(rng, (B, G * Hkv, d))
+    o = OR.default()
+    nb = -(-n // bs)
+    summ_h = np.zeros((B, Hkv, dims.maxnb, 2, d), np.uint16)
+    lohi = {}
+    for b in range(B):
+        for h in range(Hkv):
+            lo, hi = o.build_summaries(k[b, h], n, bs)
+            lohi[(b, h)] = (lo, hi)
+            summ_h[b, h, :nb, 0] = W.f32_to_bf16_bits(lo.astype(np.float32))
+            summ_h[b, h, :nb, 1] = W.f32_to_bf16_bits(hi.astype(np.float32))
+    S = dims.sel_heads
+    pred_h = np.full((B, S, K), -1, np.int32)
+    for b in range(B):
+        for s_ in range(S):
+            pred_h[b, s_] = np.sort(rng.choice(nb, size=K, replace=False))
+    ws = torch.zeros(prr.prr_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    seq = torch.full((B,), n, dtype=torch.int32, device="cuda")
+    sel = torch.zeros((B, S, K), dtype=torch.int32, device="cuda")
+    missed, nm = torch.zeros_like(sel), torch.zeros((B, S), dtype=torch.int32, device="cuda")
+    keep = torch.zeros((B, S, K), dtype=torch.uint8, device="cuda")
+    prr.prr_workspace_init(ws)
+    prr.prr_select_topk(dims, to_dev_bits(q), to_dev_bits(summ_h), seq, torch.from_numpy(pred_h).cuda(), sel, missed,
+                        nm, keep, ws)
+    torch.cuda.synchronize()
+    assert prr.prr_get_device_status(ws) == 0
+    g_sel, g_missed, g_keep = sel.cpu().numpy(), missed.cpu().numpy(), keep.cpu().numpy()
+    for b in range(B):
+        for s_ in range(S):
+            kvh, rows = (s_ // G, slice(s_, s_ + 1)) if selector == "per_head" else (s_, slice(s_ * G, (s_ + 1) * G))
+            lo, hi = lohi[(b, kvh)]
+            qg = f64(q[b, rows])
+            sc = o.block_scores_max(qg, lo, hi) if selector == "group_max" else o.block_scores(qg, lo, hi)
+            ref = o.top_ranked_forced(sc, K, n_sink, n_local) if (n_sink or n_local) else o.top_ranked(sc, K)
+            assert np.array_equal(g_sel[b, s_], pad(ref, K)), (b, s_, g_sel[b, s_].tolist(), ref.tolist())
+            ref_missed, ref_keep = o.missed_keep(ref, pred_h[b, s_])
+            assert np.array_equal(g_missed[b, s_], pad(ref_missed, K))
+            assert np.array_equal(g_keep[b, s_], ref_keep)
+    if (n_sink, n_local, K) == (2, 4, 3):
+        assert all(list(g_sel[b, s_]) == [0, 1, nb - 1] for b in range(B) for s_ in range(S))
+
+
+# ----------------------------------------------------------------------------- paged KV
+
+@pytest.mark.parametrize("mode", MODES)
+def test_decode_paged_ragged(mode):
+    """Paged KV cache (every block in its own page, pages in shuffled order behind a
+    block table) with a ragged batch; then 128-token pages with the token appended
+    inside the step and CUDA graphs."""
+    w = W.workload("tiny").with_(name="paged", B=3, Hq=8, Hkv=2, d=128, N0=2600, bs=64, K=16, P=16, steps=10,
+                                 walk_p=0.8, n0_seq=(2600, 1777, 2049))
+    _assert_ok(run_parity(w, steps=10, mode=mode, paged=True))
+    w2 = w.with_(bs=128, n0_seq=(2600, 901, 1280))
+    _assert_ok(run_parity(w2, steps=6, mode=mode, paged=True, append="step", graph=True))
+
+
+def test_decode_paged_variants():
+    """Paged KV under per-head selection with forced blocks (fused step)."""
+    w = W.workload("tiny").with_(name="paged_variant", B=2, Hq=8, Hkv=2, d=64, N0=3000, bs=64, K=12, P=12,
+                                 steps=5, walk_p=0.8, selector="per_head", n_sink=1, n_local=1, n0_seq=(3000, 2222))
+    _assert_ok(run_parity(w, steps=5, paged=True))
+
+
+def test_decode_paged_full_size():
+    """The headline 128K batched workload on a paged cache, sampled units, graphs."""
+    _assert_ok(run_parity(W.workload("batched_128k"), steps=3, units=[(0, 0), (15, 7)], graph=True, paged=True))
+
+
+def test_bad_block_table_sets_status_without_fault():
+    """A block-table entry outside the pool is reported (PRR_DEV_BAD_RANGE) and not read:
+    the tail block's entry, which the step reads to fold the newest key."""
+    w = W.workload("tiny").with_(name="paged_bad", B=1, Hq=4, Hkv=1, d=64, N0=1000, bs=64, K=4, P=4, steps=2)
+    dec, dims = make_decoder(w, 2, paged=True)
+    dec.block_table[0, (w.N0 - 1) // w.bs] = dims.pages + 5  # past the pool
+    dec.step_fused(to_dev_bits(W.queries(w, 1)[0]))
+    torch.cuda.synchronize()
+    assert dec.device_status() == 5
+
+
 # ----------------------------------------------------------------------------- device status
 
 def test_bad_seq_len_sets_status_without_fault():
@@ -355,6 +488,93 @@ def test_bad_seq_len_sets_status_without_fault():
     dec.step(to_dev_bits(W.queries(w, 1)[0]))
     torch.cuda.synchronize()
     assert dec.device_status() == 0
+
+
+def test_wait_timeout_returns_status_without_fault():
+    """A bounded wait that runs out, without a fault: the workspace test word makes the
+    fused step skip its selection chunks, so no unit's top-K completes and the launch's
+    end-of-step wait gives up after its one-second limit with PRR_DEV_WAIT_TIMEOUT (4).
+    The context stays usable: after re-initialising the workspace a normal step
+    selects the oracle's top-K and matches its attention."""
+    from tests.prr_harness import UnitOracle, compare_attention, Report
+    w = W.workload("tiny")
+    dec, dims = make_decoder(w, 4)
+    dec.ws.view(torch.int32)[prr.WS_TEST_SKIP_SELECTION_OFFSET // 4] = 1
+    q = W.queries(w, 1)
+    dec.step_fused(to_dev_bits(q[0]))
+    torch.cuda.synchronize()
+    assert dec.device_status() == 4
+    prr.prr_workspace_init(dec.ws)
+    dec.step_fused(to_dev_bits(q[0]))
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    uo = UnitOracle.create(w, 0, 0, 1, OR.default())
+    n, nb, qg, s, sel = uo.select(-1, q[0])  # no token appended: n = N0
+    assert np.array_equal(dec.sel[0, 0].cpu().numpy(), pad(sel, w.K))
+    res = uo.finish(n, nb, qg, sel, np.zeros(0, np.int32))
+    rep = Report()
+    compare_attention(rep, "after timeout", dec.out[0].cpu().numpy(), dec.lse[0].cpu().numpy(), res["out"], res["lse"])
+    assert not rep.messages, rep.messages
+
+
+def test_sharded_decoder_matches_one_decoder():
+    """Two shards of one batch (here both on cuda:0, as independent decoders that never
+    wait on each other) give the same outputs, bit for bit, as one decoder over the
+    whole batch: units are independent, so sharding needs no exchange."""
+    from dynamic_sparse_attention_block_b200.sharding import ShardedDecoder
+    w = W.workload("tiny").with_(name="shards", B=5, Hq=8, Hkv=2, d=128, N0=2000, bs=64, K=8, P=8, per_seq_seed=True)
+    steps = 4
+    one, dims = make_decoder(w, steps)
+    dev = torch.device("cuda", 0)
+    sh = ShardedDecoder(dims, [dev, dev])
+    for (b0, b1), dec in sh.shards:
+        for i, b in enumerate(range(b0, b1)):
+            for h in range(w.Hkv):
+                k0, v0 = W.kv_prefix(w, b, h)
+                dec.load_context(i, h, to_dev_bits(k0), to_dev_bits(v0))
+        dec.prefill(None, None, w.N0)
+    kn, vn = __import__("tests.gpu_runner", fromlist=["appended_tokens"]).appended_tokens(w, steps)
+    qs = W.queries(w, steps)
+    for t in range(steps):
+        q, k, v = to_dev_bits(qs[t]), to_dev_bits(kn[t]), to_dev_bits(vn[t])
+        one.step_fused(q, k_new=k, v_new=v)
+        sh.step_fused(q, k, v)
+        torch.cuda.synchronize()
+        for (b0, b1), out, lse in sh.outputs():
+            assert torch.equal(out, one.out[b0:b1]) and torch.equal(lse, one.lse[b0:b1]), (t, b0)
+    assert one.device_status() == 0 and all(d.device_status() == 0 for _, d in sh.shards)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_checkpoint_resume_bit_identical(paged):
+    """Resume: n steps, the decoder's state copied to the host and loaded into a fresh
+    decoder, m more steps -- bit-identical to n + m steps without the break (outputs,
+    selections, EMA state and predictions)."""
+    from tests.gpu_runner import appended_tokens
+    w = W.workload("tiny").with_(name="resume", B=2, Hq=8, Hkv=2, d=128, N0=3000, bs=64, K=12, P=12, steps=8,
+                                 walk_p=0.7, per_seq_seed=True)
+    n, m = 5, 3
+    kn, vn = appended_tokens(w, n + m)
+    qs = W.queries(w, n + m)
+
+    def run(dec, t0, t1):
+        for t in range(t0, t1):
+            dec.step_fused(to_dev_bits(qs[t]), k_new=to_dev_bits(kn[t]), v_new=to_dev_bits(vn[t]))
+        torch.cuda.synchronize()
+
+    a, _ = make_decoder(w, n + m, paged=paged)
+    run(a, 0, n + m)
+    b, _ = make_decoder(w, n + m, paged=paged)
+    run(b, 0, n)
+    ck = b.checkpoint()
+    del b
+    c, _ = make_decoder(w, n + m, paged=paged)
+    c.restore(ck)
+    run(c, n, n + m)
+    for name in ("out", "lse", "sel", "missed", "ema", "seq_lens", "summ"):
+        assert torch.equal(getattr(a, name), getattr(c, name)), name
+    assert torch.equal(a.pred, c.pred)
+    assert a.device_status() == 0 and c.device_status() == 0
 
 
 def test_bad_pred_sets_status_without_fault():

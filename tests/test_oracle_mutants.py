@@ -37,6 +37,11 @@ MUTANTS = [
     ("variant_max_takes_min", "if (h == 0 || u > best) best = u;", "if (h == 0 || u < best) best = u;"),
     ("variant_first_sink_skipped", "for (int b = 0; b < n_sink", "for (int b = 1; b < n_sink"),
     ("variant_local_from_oldest", "int b = nb - 1 - i;", "int b = i;"),
+    ("rep_offset_ignored", "const uint16_t *krow = k + ((size_t)b * bs + off) * d;",
+     "const uint16_t *krow = k + ((size_t)b * bs) * d;"),
+    ("paged_wrong_head", "((size_t)table[t / bs] * Hkv + h) * bs", "((size_t)table[t / bs] * Hkv) * bs"),
+    ("paged_block_not_mapped", "((size_t)table[t / bs] * Hkv + h) * bs", "((size_t)(t / bs) * Hkv + h) * bs"),
+    ("rep_tail_not_clamped", "if (off > valid - 1) off = valid - 1;", "if (off > bs - 1) off = bs - 1;"),
 ]
 
 

@@ -33,6 +33,14 @@ def _bits(rng, shape, gauss):
     return torch.from_numpy(W.f32_to_bf16_bits(np.asarray(x, np.float32)).view(np.int16)).cuda()
 
 
+def _summaries(rng, B, Hkv, maxnb, d, gauss):
+    """Valid block summaries: per channel a min row not above the max row (the scorer's
+    bound equals the oracle's only for such pairs)."""
+    x = rng.standard_normal((B, Hkv, maxnb, 2, d)) if gauss else rng.integers(-8, 9, size=(B, Hkv, maxnb, 2, d)) / 8
+    x = np.sort(x, axis=3)
+    return torch.from_numpy(W.f32_to_bf16_bits(np.asarray(x, np.float32)).view(np.int16)).cuda()
+
+
 def _outputs(B, Hkv, K, P):
     sel = torch.full((B, Hkv, K), -7, dtype=torch.int32, device="cuda")
     return (sel, torch.full_like(sel, -7), torch.full((B, Hkv), -7, dtype=torch.int32, device="cuda"),
@@ -54,7 +62,7 @@ def test_static_scratch_matches_workspace_entry(d, bs, G, K, P, n, gauss):
     seq = torch.full((B,), n, dtype=torch.int32, device="cuda")
     status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for call in range(2):  # fresh inputs each call: the shared array keeps the last call's contents
-        summ = _bits(rng, (B, Hkv, dims.maxnb, 2, d), gauss)
+        summ = _summaries(rng, B, Hkv, dims.maxnb, d, gauss)
         q = _bits(rng, (B, G * Hkv, d), gauss)
         pred_h = np.full((B, Hkv, max(P, 1)), -1, np.int32)
         for b in range(B):
@@ -106,7 +114,7 @@ def test_static_scratch_recovers_after_bad_seq_len():
     cap = n + 3
     dims = prr.Dims(B=B, Hq=G * Hkv, Hkv=Hkv, d=d, bs=bs, cap_tokens=cap, K=K, P=P)
     nb = -(-n // bs)
-    summ = _bits(rng, (B, Hkv, dims.maxnb, 2, d), False)
+    summ = _summaries(rng, B, Hkv, dims.maxnb, d, False)
     q = _bits(rng, (B, G * Hkv, d), False)
     pred_h = np.full((B, Hkv, P), -1, np.int32)
     for b in range(B):

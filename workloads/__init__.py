@@ -59,14 +59,27 @@ class Workload:
     per_seq_seed: bool = False
     seed: int = 0
     forced_overlaps: Optional[Sequence[float]] = None  # forced predictor overlap levels
+    selector: str = "group_sum"  # block selector: "group_sum", "group_max" or "per_head"
+    n_sink: int = 0              # forced first blocks
+    n_local: int = 0             # forced newest blocks
+    n0_seq: Optional[Sequence[int]] = None  # ragged batch: context of each sequence (each <= N0)
 
     @property
     def G(self) -> int:
         return self.Hq // self.Hkv
 
     @property
+    def sel_heads(self) -> int:
+        """Selections per sequence: KV heads, or query heads under per-head selection."""
+        return self.Hq if self.selector == "per_head" else self.Hkv
+
+    @property
     def units(self) -> int:
-        return self.B * self.Hkv
+        return self.B * self.sel_heads
+
+    def n0(self, b: int) -> int:
+        """Context length of sequence b before the first decode step."""
+        return self.n0_seq[b] if self.n0_seq is not None else self.N0
 
     def seed_of(self, b: int) -> int:
         # per-sequence seeds are b (plus an offset that distinguishes replicas)
