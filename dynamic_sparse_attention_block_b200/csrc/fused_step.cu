@@ -323,7 +323,17 @@ __device__ bool prod_emit(const Params& p, const FusedSmem& S, const CUtensorMap
   if (use > 0 && !mbar_wait_idle(&S.empty[s], (use - 1) & 1u, p.status)) return false;
   unsigned char* slot = S.slots + static_cast<size_t>(s) * p.fslot_bytes;
   unsigned char* aux = S.aux + static_cast<size_t>(s) * kAuxBytes;
+#ifdef PRR_PHASE_DEBUG
+  {
+    ItemDesc d = it;
+    const unsigned long long now = global_ns();
+    d.pad[0] = static_cast<int>(now & 0xFFFFFFFFu);
+    d.pad[1] = static_cast<int>(now >> 32);
+    *reinterpret_cast<ItemDesc*>(aux + kAuxDesc) = d;
+  }
+#else
   *reinterpret_cast<ItemDesc*>(aux + kAuxDesc) = it;
+#endif
   const uint32_t qbytes = static_cast<uint32_t>(p.G) * D * 2;
   const uint16_t* qsrc = p.q + static_cast<size_t>(it.u) * p.G * D;
   fence_proxy_async();  // the consumers' generic writes to this slot precede the new copies
@@ -437,6 +447,28 @@ __device__ void producer(const Params& p, const FusedCtl& C, const FusedSmem& S,
     if (__shfl_sync(kFull, abort_seen, 0)) {
       ok = false;
       break;
+    }
+    // Start the batch's tiles towards L2 now: the ring takes them a few items later, and
+    // by then their copies into shared memory come from L2, so a slot's wait for its
+    // data -- and the time the ring spends not streaming -- is short.
+    if (static_cast<unsigned>(lane) < cnt && emit) {
+      if (mine.kind == kItemSel) {
+        const int c0 = mine.idx * p.fchunk_blocks;
+        const int rows = max(0, min(p.fchunk_blocks, p.maxnb - c0));
+        if (rows > 0)
+          prefetch_l2(p.summ + (static_cast<size_t>(mine.u / p.kv_div) * p.maxnb + c0) * 2 * D,
+                      static_cast<uint32_t>(rows) * 4 * D);
+      } else {
+        int tok0;
+        const int slice = kv_tile(p, mine.u / p.kv_div, mine.blk, &tok0);
+        if (!p.table || slice < p.pages * p.Hkv) {  // (a bad block-table entry is not prefetched)
+#pragma unroll
+          for (int r = 0; r < D / 64; ++r) {
+            prefetch_l2_tile_3d(kmap, r * 64, tok0, slice);
+            prefetch_l2_tile_3d(vmap, r * 64, tok0, slice);
+          }
+        }
+      }
     }
 
     // ---- the claimed queue entry first (repairs and merges are on the critical path)
@@ -570,6 +602,17 @@ __device__ void consumer(const Params& p, const FusedCtl& C, const FusedSmem& S,
       if (tid == 0) resolve_count(p, C, pc);
       return;
     }
+#ifdef PRR_PHASE_DEBUG
+    unsigned long long* dbg_item =
+        (it.trace >= 0 && it.trace < (1 << 16)) ? g_item[it.trace] : nullptr;
+    if (dbg_item && tid == 0) {
+      dbg_item[0] = (static_cast<unsigned long long>(static_cast<unsigned>(it.pad[1])) << 32) |
+                    static_cast<unsigned>(it.pad[0]);
+      dbg_item[1] = global_ns();
+    }
+#else
+    unsigned long long* dbg_item = nullptr;
+#endif
     if (p.trace && tid == 0) {
       unsigned smid;
       asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
@@ -607,9 +650,18 @@ __device__ void consumer(const Params& p, const FusedCtl& C, const FusedSmem& S,
       const uint16_t* pk = tail_new ? p.k_new + kvrow : nullptr;
       const uint16_t* pv = tail_new ? p.v_new + kvrow : nullptr;
       if (it.blk >= 0 && it.blk < (it.n + BS - 1) / BS) {
+        // the slot goes back as soon as the tiles are read, before the partial is written
         ok = attn_compute<D, BS>(p, reinterpret_cast<const uint16_t*>(aux + kAuxQ), it.blk, it.n, dst, slot,
                                  slot + L::TILEB, reinterpret_cast<float*>(aux + kAuxRed), &S.fullK[s],
-                                 &S.fullV[s], ph, grp, pk, pv);
+                                 &S.fullV[s], ph, grp,
+                                 [&] {
+                                   released = true;
+                                   if (tid == 0) {
+                                     mbar_arrive(&S.empty[s]);
+                                     if (dbg_item) dbg_item[3] = global_ns();
+                                   }
+                                 },
+                                 pk, pv, dbg_item ? dbg_item + 2 : nullptr);
       } else {  // a missed entry out of range: contribute nothing (copies still land)
         if (tid == 0) {
           report(p.status, kDevBadMissed);
@@ -618,11 +670,14 @@ __device__ void consumer(const Params& p, const FusedCtl& C, const FusedSmem& S,
         write_empty_partial(dst, p.G, D, grp);
       }
       if (ok) {
-        fence_proxy_async();  // generic writes to the tiles precede the copies that refill them
-        gsync(grp);           // the partial is written and the slot is no longer read
-        released = true;
+        if (!released) {  // (the out-of-range path did not hand the slot back yet)
+          fence_proxy_async();
+          gsync(grp);
+          released = true;
+          if (tid == 0) mbar_arrive(&S.empty[s]);
+        }
+        gsync(grp);  // every thread's partial precedes the count
         if (tid == 0) {
-          mbar_arrive(&S.empty[s]);
           bump(p.stats, spec ? kStatSpecAttended : kStatRepaired);
           resolve_count(p, C, pc);         // the previous item's count has long returned
           pc = issue_count(C, it.u, 1u);   // looked at before the next wait or item end
@@ -762,5 +817,9 @@ size_t fused_ctl_words_for(int units, int P, int K, int G) { return fused_ctl_wo
 // Debug builds only: copy the per-unit phase timestamps of the finisher and predictor.
 extern "C" int prr_debug_phases(void* dst) {
   return static_cast<int>(cudaMemcpyFromSymbol(dst, prr::g_phase, sizeof(prr::g_phase)));
+}
+
+extern "C" int prr_debug_items(void* dst) {
+  return static_cast<int>(cudaMemcpyFromSymbol(dst, prr::g_item, sizeof(prr::g_item)));
 }
 #endif

@@ -15,10 +15,11 @@
 // heads.  Both products run on the tensor cores with mma.m16n8k16 in swap-AB form:
 //   S^T[tok][h] = K[tok][:] . Q^T[:][h]     (M = 16 tokens, N = 8 heads, K = d)
 //   O^T[c][h]   = V^T[c][tok] . P^T[tok][h] (M = 16 channels, N = 8 heads, K = tokens)
-// The S^T accumulator fragment becomes the P^T operand fragment through movmatrix
-// (an in-register 8x8 transpose).  P is split as bf16 hi + bf16 lo (two MMAs) so the
-// PV product keeps ~16 mantissa bits.  Four warps own disjoint token slices; their O^T
-// partial sums are added in shared memory.
+// P is split as bf16 hi + bf16 lo (two MMAs) so the PV product keeps ~16 mantissa
+// bits.  For S^T and the softmax the four warps own token slices; P goes through a
+// small buffer in the dead K tile, and for O^T they own channel slices over all
+// tokens, so each warp finishes whole output columns and the tiles are free before the
+// partial is written out.
 //
 // The copies and the arithmetic are separate steps (attn_issue, attn_compute): the
 // standalone kernels run both in one CTA; the fused step's producer warp issues the
@@ -89,16 +90,27 @@ __device__ __forceinline__ void tile_put_row(unsigned char* tile, int r, const u
 // mbarriers, waited on with parity `phase` (bounded).  When `patch_k` is not null, the
 // token n-1 (which lies in this block) is taken from patch_k / patch_v instead of the
 // staged tiles (the caller has not written it to the cache yet).  `red` is 80 floats of
-// shared scratch.  Returns false if a copy did not land in time (status word set).
-template <int D, int BS>
+// shared scratch.  tiles_free() is called by every thread once no thread reads the
+// tiles any more -- before the partial is written out -- so a caller can hand the
+// buffers back early.  Returns false if a copy did not land in time (status word set;
+// tiles_free is then not called).
+//
+// Work split: for S^T and the softmax each warp owns a slice of the tokens; P (bf16
+// high and low parts) then goes through a small buffer in the dead K tile, and for
+// O^T = V^T P^T each warp owns a slice of the channels over all tokens, so every warp
+// finishes whole output columns and no cross-warp sum of O is needed.
+template <int D, int BS, typename TilesFree>
 __device__ bool attn_compute(const Params& p, const uint16_t* q, int blk, int n, const PartialDst& dst,
                              unsigned char* sK, unsigned char* sV, float* red, uint64_t* barK, uint64_t* barV,
-                             uint32_t phase, const Grp& grp, const uint16_t* patch_k = nullptr,
-                             const uint16_t* patch_v = nullptr) {
+                             uint32_t phase, const Grp& grp, TilesFree tiles_free, const uint16_t* patch_k = nullptr,
+                             const uint16_t* patch_v = nullptr, unsigned long long* t_v = nullptr) {
   using L = AttnTile<D, BS>;
   constexpr int REGB = L::REGB, NREG = D / 64;
-  constexpr int MTW = BS / 64;  // 16-token m-tiles per warp (4 warps)
+  constexpr int MTW = BS / 64;  // 16-token m-tiles per warp for S^T (4 warps)
   constexpr int KS = D / 16;    // k-steps of QK^T == 16-channel tiles of PV
+  constexpr int CT = KS / 4;    // 16-channel tiles per warp for O^T
+  constexpr int PST = BS + 8;   // row stride (bf16) of the P buffer; the pad spreads rows over banks
+  static_assert(2 * 8 * PST * 2 <= L::TILEB, "P buffer fits in the K tile");
   const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
   const int G = p.G;
 
@@ -126,7 +138,7 @@ __device__ bool attn_compute(const Params& p, const uint16_t* q, int blk, int n,
     gsync(grp);
   }
 
-  // ---- S^T = K Q^T on the tensor cores
+  // ---- S^T = K Q^T on the tensor cores (this warp's tokens)
   const uint32_t sK_addr = smem_addr(sK), sV_addr = smem_addr(sV);
   float sc[MTW][4];
 #pragma unroll
@@ -166,7 +178,7 @@ __device__ bool attn_compute(const Params& p, const uint16_t* q, int blk, int n,
     red[warp * 8 + 2 * t] = mx0;
     red[warp * 8 + 2 * t + 1] = mx1;
   }
-  gsync(grp);
+  gsync(grp);  // the maxima are visible, and every warp is past its reads of the K tile
   float m0 = red[2 * t], m1 = red[2 * t + 1];
 #pragma unroll
   for (int w = 1; w < 4; ++w) {
@@ -174,22 +186,25 @@ __device__ bool attn_compute(const Params& p, const uint16_t* q, int blk, int n,
     m1 = fmaxf(m1, red[w * 8 + 2 * t + 1]);
   }
 
-  // ---- P = 2^(s - m), split hi/lo, transposed into B fragments
+  // ---- P = 2^(s - m) as bf16 high + low parts, [head][token] in the dead K tile
+  uint16_t* Ph = reinterpret_cast<uint16_t*>(sK);
+  uint16_t* Pl = Ph + 8 * PST;
   float ls0 = 0.f, ls1 = 0.f;
-  uint32_t bh[MTW][2], bl[MTW][2];
 #pragma unroll
   for (int mi = 0; mi < MTW; ++mi) {
-    const float p0 = exp2f(sc[mi][0] - m0), p1 = exp2f(sc[mi][1] - m1);
-    const float p2 = exp2f(sc[mi][2] - m0), p3 = exp2f(sc[mi][3] - m1);
-    ls0 += p0 + p2;
-    ls1 += p1 + p3;
-    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
-    const uint32_t l01 = pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01));
-    const uint32_t l23 = pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23));
-    bh[mi][0] = movmatrix_trans(h01);
-    bh[mi][1] = movmatrix_trans(h23);
-    bl[mi][0] = movmatrix_trans(l01);
-    bl[mi][1] = movmatrix_trans(l23);
+    const int tok = (warp * MTW + mi) * 16 + g;
+    const float pv[4] = {exp2f(sc[mi][0] - m0), exp2f(sc[mi][1] - m1), exp2f(sc[mi][2] - m0),
+                         exp2f(sc[mi][3] - m1)};
+    ls0 += pv[0] + pv[2];
+    ls1 += pv[1] + pv[3];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int h = 2 * t + (e & 1), tk = tok + (e >> 1) * 8;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(pv[e]);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(pv[e] - __bfloat162float(hi));
+      Ph[h * PST + tk] = __bfloat16_as_ushort(hi);
+      Pl[h * PST + tk] = __bfloat16_as_ushort(lo);
+    }
   }
 #pragma unroll
   for (int o = 4; o <= 16; o <<= 1) {
@@ -201,7 +216,8 @@ __device__ bool attn_compute(const Params& p, const uint16_t* q, int blk, int n,
     red[32 + warp * 8 + 2 * t + 1] = ls1;
   }
 
-  if (!gsync_and(grp, mbar_wait(barV, phase, p.status))) return false;
+  if (!gsync_and(grp, mbar_wait(barV, phase, p.status))) return false;  // also publishes P
+  if (t_v && tid == 0) *t_v = global_ns();  // debug timelines: the V tile is usable
   if (nv < BS) {  // tokens past the end of the sequence: zero V so 0 * V stays 0
     uint4* v4 = reinterpret_cast<uint4*>(sV);
     const int rows = BS - nv;
@@ -225,55 +241,49 @@ __device__ bool attn_compute(const Params& p, const uint16_t* q, int blk, int n,
     red[72 + 2 * t + 1] = l1;
   }
 
-  // ---- O^T = V^T P^T on the tensor cores
-  float oacc[KS][4];
+  // ---- O^T = V^T P^T on the tensor cores (this warp's channels, all tokens)
+  float oacc[CT][4];
 #pragma unroll
-  for (int dt = 0; dt < KS; ++dt) oacc[dt][0] = oacc[dt][1] = oacc[dt][2] = oacc[dt][3] = 0.f;
+  for (int ct = 0; ct < CT; ++ct) oacc[ct][0] = oacc[ct][1] = oacc[ct][2] = oacc[ct][3] = 0.f;
+  const uint32_t pb_addr = smem_addr(((lane >> 4) ? Pl : Ph) + (lane & 7) * PST + ((lane >> 3) & 1) * 8);
 #pragma unroll
-  for (int mi = 0; mi < MTW; ++mi) {
-    const int mt = warp * MTW + mi;
-    const int row = mt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+  for (int kt = 0; kt < BS / 16; ++kt) {
+    uint32_t b[4];  // P^T fragments of tokens 16kt..: high part (k 0-7, 8-15), low part
+    ldsm_x4(pb_addr + kt * 32, b);
+    const int row = kt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
 #pragma unroll
-    for (int dt = 0; dt < KS; ++dt) {
+    for (int ct = 0; ct < CT; ++ct) {
+      const int dt = warp * CT + ct;
       const int ch = 2 * dt + ((lane >> 3) & 1);
       const uint32_t addr = sV_addr + (ch >> 3) * REGB + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
       uint32_t a[4];
       ldsm_x4_trans(addr, a);
-      mma_16816(oacc[dt], a, bh[mi][0], bh[mi][1]);
-      mma_16816(oacc[dt], a, bl[mi][0], bl[mi][1]);
+      mma_16816(oacc[ct], a, b[0], b[1]);
+      mma_16816(oacc[ct], a, b[2], b[3]);
     }
   }
-  // per-warp O^T into the (dead) K tile: redO[warp][h][c ^ 4h], conflict-free (every
-  // warp passed a group barrier after its last K-tile read)
-  float* redO = reinterpret_cast<float*>(sK);
+  fence_proxy_async();  // this thread's generic writes to the tiles precede later copies
+  gsync(grp);           // no thread reads the tiles any more
+  tiles_free();
+
+  // ---- the partial: whole columns from each warp, m and l from the reductions
 #pragma unroll
-  for (int dt = 0; dt < KS; ++dt) {
-    const int c0 = dt * 16 + g;
-    redO[(warp * 8 + 2 * t) * D + (c0 ^ (8 * t))] = oacc[dt][0];
-    redO[(warp * 8 + 2 * t + 1) * D + (c0 ^ (8 * t + 4))] = oacc[dt][1];
-    redO[(warp * 8 + 2 * t) * D + ((c0 + 8) ^ (8 * t))] = oacc[dt][2];
-    redO[(warp * 8 + 2 * t + 1) * D + ((c0 + 8) ^ (8 * t + 4))] = oacc[dt][3];
-  }
-  gsync(grp);
-  constexpr int C4 = D / 4;
-  for (int e = tid; e < G * C4; e += grp.nt) {
-    const int h = e / C4, c4 = e % C4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float4 v = *reinterpret_cast<const float4*>(redO + (w * 8 + h) * D + ((4 * c4) ^ (4 * h)));
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+  for (int ct = 0; ct < CT; ++ct) {
+    const int c0 = (warp * CT + ct) * 16 + g;
+    const int h0 = 2 * t, h1 = 2 * t + 1;
+    if (h0 < G) {
+      dst.O[h0 * dst.ostride + c0] = oacc[ct][0];
+      dst.O[h0 * dst.ostride + c0 + 8] = oacc[ct][2];
     }
-    reinterpret_cast<float4*>(dst.O + h * dst.ostride)[c4] = acc;
+    if (h1 < G) {
+      dst.O[h1 * dst.ostride + c0] = oacc[ct][1];
+      dst.O[h1 * dst.ostride + c0 + 8] = oacc[ct][3];
+    }
   }
   if (tid < G) {
     dst.m[tid * dst.rstride] = red[64 + tid];
     dst.l[tid * dst.rstride] = red[72 + tid];
   }
-  fence_proxy_async();  // this thread's generic writes to the tiles precede later copies
   return true;
 }
 
@@ -293,7 +303,8 @@ __device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CU
     attn_issue<D, BS>(kmap, vmap, slice, tok0, sK, sV, &bars[0], &bars[1]);
   }
   return attn_compute<D, BS>(p, p.q + static_cast<size_t>(u) * p.G * D, blk, n, dst, sK, sV,
-                             reinterpret_cast<float*>(smem + 2 * L::TILEB), &bars[0], &bars[1], phase, grp);
+                             reinterpret_cast<float*>(smem + 2 * L::TILEB), &bars[0], &bars[1], phase, grp,
+                             [] {});
 }
 
 }  // namespace prr

@@ -11,8 +11,10 @@
 namespace prr {
 
 #ifdef PRR_PHASE_DEBUG
-// Debug builds only: per-unit phase timestamps of the finisher / predictor.
+// Debug builds only: per-unit phase timestamps of the finisher / predictor, and per
+// fused item {copies issued, K landed, V landed, slot handed back}.
 __device__ unsigned long long g_phase[2][4096][8];
+__device__ unsigned long long g_item[1 << 16][4];
 #define PRR_PHASE(kind, u, k) \
   do {                        \
     if ((threadIdx.x & 127) == 0 && (u) < 4096) g_phase[kind][u][k] = global_ns(); \
@@ -225,21 +227,10 @@ __device__ __forceinline__ void fold_tail_row(uint32_t* row, const uint16_t* new
 // largest key and the mask of the blocks holding it.  From those alone the finisher
 // sees whether at least K_eff blocks tie at the overall maximum; then T is that maximum
 // and S is the first K_eff set bits of the maximal groups' masks -- no key is loaded
-// (this is the usual case when every block's bound saturates).  Otherwise one warp
-// finds T bit by bit from the most significant bit that the smallest and largest keys
-// differ in: T keeps a bit when at least K_eff keys are >= the candidate value.  That
-// needs no CTA barrier per step.
+// (this is the usual case when every block's bound saturates).  Otherwise T comes from
+// a radix selection over the keys by the whole group (radix_kth_largest).
 
-constexpr int kBitRegs = 32;     // keys per lane kept in registers by the bit search (nb <= 1024)
 constexpr int kEagerKeys = 4096;  // up to this many keys are fetched with the group summaries
-
-// Start of the bit search: the bits that the smallest and largest keys share, lower
-// bits zero (every key is >= it).
-__device__ __forceinline__ uint32_t bit_search_start(uint32_t lo, uint32_t hi) {
-  if (lo == hi) return hi;
-  const int top = 31 - __clz(lo ^ hi);  // highest differing bit
-  return top == 31 ? 0u : (hi & ~((2u << top) - 1u));
-}
 
 // One warp (all lanes): summary of the warp's group of 32 blocks (`valid` lanes).
 __device__ __forceinline__ void write_group_summary(const Params& p, int u, int group, uint32_t key, bool valid) {
@@ -340,83 +331,14 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
         have_keys = true;
         gsync(grp);
       }
-      if (warp == 0) {  // T bit by bit; every candidate count is one warp reduction
-        uint32_t t, gt;
-        if (nb <= 32 * kBitRegs) {
-          // keys held in registers (padding 0 is below every candidate, which is > 0)
-          uint32_t kr[kBitRegs];
-#pragma unroll
-          for (int q = 0; q < kBitRegs; ++q) {
-            const int i = q * 32 + lane;
-            kr[q] = i < nb ? skeys[i] : 0u;
-          }
-          uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-#pragma unroll
-          for (int q = 0; q < kBitRegs; ++q) {
-            if (q * 32 + lane < nb) lo = min(lo, kr[q]);
-            hi = max(hi, kr[q]);
-          }
-          lo = __reduce_min_sync(kFull, lo);
-          hi = __reduce_max_sync(kFull, hi);
-          t = bit_search_start(lo, hi);
-          if (lo != hi) {
-            int bit = 31 - __clz(lo ^ hi);
-            // two bits per round: three candidate counts, reduced independently
-            for (; bit >= 1; bit -= 2) {
-              const uint32_t c1 = t | (1u << (bit - 1)), c2 = t | (2u << (bit - 1)), c3 = t | (3u << (bit - 1));
-              int n1 = 0, n2 = 0, n3 = 0;
-#pragma unroll
-              for (int q = 0; q < kBitRegs; ++q) {
-                n1 += kr[q] >= c1 ? 1 : 0;
-                n2 += kr[q] >= c2 ? 1 : 0;
-                n3 += kr[q] >= c3 ? 1 : 0;
-              }
-              const int s1 = __reduce_add_sync(kFull, n1), s2 = __reduce_add_sync(kFull, n2);
-              const int s3 = __reduce_add_sync(kFull, n3);
-              t = s3 >= keff ? c3 : (s2 >= keff ? c2 : (s1 >= keff ? c1 : t));
-            }
-            if (bit == 0) {
-              const uint32_t c = t | 1u;
-              int n1 = 0;
-#pragma unroll
-              for (int q = 0; q < kBitRegs; ++q) n1 += kr[q] >= c ? 1 : 0;
-              if (__reduce_add_sync(kFull, n1) >= keff) t = c;
-            }
-          }
-          int g = 0;
-#pragma unroll
-          for (int q = 0; q < kBitRegs; ++q) g += kr[q] > t ? 1 : 0;
-          gt = __reduce_add_sync(kFull, g);
-        } else {
-          uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-          for (int i = lane; i < nb; i += 32) {
-            lo = min(lo, skeys[i]);
-            hi = max(hi, skeys[i]);
-          }
-          lo = __reduce_min_sync(kFull, lo);
-          hi = __reduce_max_sync(kFull, hi);
-          t = bit_search_start(lo, hi);
-          if (lo != hi) {
-            for (int bit = 31 - __clz(lo ^ hi); bit >= 0; --bit) {
-              const uint32_t c = t | (1u << bit);
-              int cnt = 0;
-#pragma unroll 8
-              for (int i = lane; i < nb; i += 32) cnt += skeys[i] >= c ? 1 : 0;
-              if (__reduce_add_sync(kFull, cnt) >= static_cast<unsigned>(keff)) t = c;
-            }
-          }
-          int g = 0;
-          for (int i = lane; i < nb; i += 32) g += skeys[i] > t ? 1 : 0;
-          gt = __reduce_add_sync(kFull, g);
-        }
-        if (lane == 0) {
-          ms[8] = t;
-          misc[9] = static_cast<int>(gt);
-        }
-      }
-      gsync(grp);
-      T = ms[8];
-      n_gt = misc[9];
+      // T: the K_eff-th largest key, by radix selection over the whole group (8-bit
+      // digits from the first byte the keys differ in; lanes of a warp that fall in the
+      // same bin add in one atomic, so ties at the threshold stay cheap)
+      unsigned* hist = reinterpret_cast<unsigned*>(scratch);  // first 1 KB of the scratch
+      int gt = 0;
+      T = radix_kth_largest(
+          nb, keff, [&](int i) { return skeys[i]; }, [](int) { return true; }, hist, misc + 10, &gt, grp);
+      n_gt = gt;
     }
   }
   PRR_PHASE(0, u, 2);
