@@ -1,30 +1,37 @@
 // fused_step.cu -- the whole PRR decode step in ONE persistent, warp-specialised launch.
 //
 // This is the PRR runtime (abstract; method summary; contributions (1)-(3)) scheduled
-// as a dataflow over a 148-SM part.  One CTA per SM: a producer warp and two consumer
-// groups of four warps share a ring of item slots in shared memory.
+// as a dataflow over a 148-SM part.  One CTA per SM: a producer warp, two consumer
+// groups of four warps and a bookkeeper warp share a ring of item slots in shared
+// memory.
 //
 //  * The producer takes work, resolves what each item needs to load, and issues the
 //    copies (1-D bulk copies for summary rows and query rows, 3-D TMA for K/V tiles)
 //    into the next free slot, up to a full ring ahead of the consumers, so every SM
 //    keeps several items' bytes in flight while the consumers compute.
-//  * Work comes from two places.  Main tickets (one atomic counter, claimed in
+//  * Work comes from three places.  This CTA's FINISH mailbox (taken first); the ready
+//    queue in the workspace: REPAIR (unit, missed slot, block), EMA (unit) and COMBINE
+//    (unit, query head); and the main tickets (one atomic counter, claimed in small
 //    batches): first every selection chunk (SEL: unit, 32-128 blocks), then every
-//    speculative slot (SPEC: unit, predicted slot j).  Ready tasks (a queue in the
-//    workspace, taken first): REPAIR (unit, missed slot, block), EMA (unit) and
-//    COMBINE (unit, query head).  No item ever waits for another: a task is queued
-//    only once everything it reads exists.
-//  * SEL folds the appended key into its block's summary (a1), scores the chunk's
-//    blocks (a2) and counts the chunk done.  The consumer that scores a unit's last
-//    chunk runs the top-K finisher (a3) right away, publishes S_t, M_t = S_t \ Pred_t
-//    and the keep mask, and queues one REPAIR per missed block plus the unit's EMA
-//    update (a4).
-//  * SPEC attends one predicted block (a5); a predicted block that selection has
-//    already dropped is skipped by the producer (its partial would be discarded).
-//    REPAIR attends one missed block (a6).  Each unit counts its finished partials;
-//    the finisher adds (large constant - expected count), so whichever partial or
-//    finisher completes the count queues the unit's COMBINE tasks: the LSE merge of
-//    the kept speculative and the repair partials (a6).
+//    speculative slot (SPEC: unit, predicted slot j).  No item ever waits for
+//    another: a task exists only once everything it reads does.
+//  * SEL folds the appended key into its block's summary (a1) and scores the chunk's
+//    blocks (a2).  FINISH runs a unit's top-K (a3) once all its chunks are scored,
+//    publishes S_t, M_t = S_t \ Pred_t and the keep mask, and queues one REPAIR per
+//    missed block (a4).  SPEC attends one predicted block (a5); a predicted block that
+//    selection has already dropped is skipped by the producer.  REPAIR attends one
+//    missed block (a6); COMBINE is the LSE merge of one query head (a6); EMA is the
+//    unit's predictor update (a4).
+//  * Consumers never wait on global memory ordering.  Whatever must be published to
+//    other CTAs with release semantics -- a chunk scored, a partial written, a
+//    finisher's outputs, a merge or predictor update done -- a consumer group posts as
+//    a record to the bookkeeper warp through shared memory.  The bookkeeper takes the
+//    records in batches: one release fence covers all of them, then the counter
+//    updates (one lane each), then, for the counts that complete, one acquire fence
+//    and the follow-up tasks: FINISH into this CTA's mailbox when a unit's last chunk
+//    is counted, the unit's EMA task when its finisher is done, and its COMBINE tasks
+//    when its partial count completes (the finisher adds a large constant minus the
+//    expected count, so whichever add lands last completes it).
 //  * The launch ends when every unit's merges and predictor update are done; the
 //    producers then send their consumer groups an exit item.
 //
@@ -49,8 +56,9 @@
 
 namespace prr {
 
-constexpr int kFusedThreads = 288;       // two consumer groups of 128 + one producer warp
+constexpr int kFusedThreads = 320;       // two consumer groups of 128, a producer and a bookkeeper warp
 constexpr int kProducerWarp = 8;
+constexpr int kBookWarp = 9;
 constexpr int kAuxBytes = 4096;          // per slot: q rows, key row, reductions, descriptor
 constexpr int kAuxQ = 0;                 // G*D bf16 query rows (<= 2048 bytes)
 constexpr int kAuxNewK = 3072;           // the appended key row (D bf16)
@@ -70,18 +78,23 @@ enum : int {
   kCtlUnits = 16,    // per-unit words start here
 };
 
-enum : int { kItemExit = 0, kItemSel = 1, kItemSpec = 2, kItemRepair = 3, kItemEma = 4, kItemCombine = 5 };
+enum : int {
+  kItemExit = 0, kItemSel = 1, kItemSpec = 2, kItemRepair = 3, kItemEma = 4, kItemCombine = 5, kItemFinish = 6
+};
 
 // What a consumer finds in its slot.
 struct ItemDesc {
   int kind;
-  int u;      // unit
-  int idx;    // SEL: chunk; SPEC: predicted slot; REPAIR: missed slot; COMBINE: query head
-  int blk;    // SPEC / REPAIR: block
-  int n;      // tokens of the unit's sequence this step (0 if seq_lens was invalid)
-  int trace;  // trace record index
-  int pad[2];
+  int u;          // unit
+  int idx;        // SEL: chunk; SPEC: predicted slot; REPAIR: missed slot; COMBINE: query head
+  int blk;        // SPEC / REPAIR: block
+  int n;          // tokens of the unit's sequence this step (0 if seq_lens was invalid)
+  int trace;      // trace record index
+  unsigned seq;   // ring sequence number of this use of the slot
+  unsigned pad;
+  unsigned long long t_issue;  // debug builds: when the copies were issued
 };
+constexpr unsigned kNoSeq = 0xFFFFFFFFu;  // a slot's descriptor before its first use
 
 struct FusedCtl {
   unsigned* words;          // the fixed words above
@@ -133,57 +146,69 @@ size_t fused_slot_bytes(const Params& p) {
   return (b + 1023) & ~static_cast<size_t>(1023);
 }
 
-// ---------------------------------------------------------------- queue helpers
+// ---------------------------------------------------------------- ready queue
 // Tasks are appended by reserving entries (atomic add on the tail) and publishing each
-// word with a release store, so a taker that reads the word non-zero also sees what
-// the task reads.  Takers claim entry indices one at a time with an atomic add on the
-// head (no compare-and-swap retries, so many idle CTAs do not contend): a claimed index
-// may lie ahead of the tail, and the claimer checks it without blocking until a task
-// lands there or the step is over.
+// word with a store that follows a release fence (or needs none: a repair's word is all
+// it reads), so a taker that reads the word non-zero also sees what the task reads.
+// Takers claim entry indices one at a time with an atomic add on the head (no
+// compare-and-swap retries, so many idle CTAs do not contend): a claimed index may lie
+// ahead of the tail, and the claimer checks it without blocking until a task lands
+// there or the step is over.
 
-// One thread: append `cnt` task words.
-__device__ inline void rq_push(const Params& p, const FusedCtl& C, const unsigned long long* tasks, int cnt) {
-  const unsigned pos = atomicAdd(C.words + kCtlRqTail, static_cast<unsigned>(cnt));
-  for (int i = 0; i < cnt; ++i) {
-    if (pos + i < static_cast<unsigned>(p.rq_cap)) {
-      st_release64(C.rq + pos + i, tasks[i]);
-    } else {
-      report(p.status, kDevWaitTimeout);  // cannot happen: the queue holds every task of a step
-      atomicExch(C.words + kCtlAbort, 1u);
-    }
-  }
-}
+// ---------------------------------------------------------------- bookkeeping records
+// A record is one 64-bit word: op (bits 56-63), unit (32-55), argument (0-31).  Three
+// single-writer rings (consumer group 0, group 1, producer) feed the bookkeeper warp.
+enum : unsigned {
+  kRecSelDone = 1,   // a SEL chunk of the unit is scored (keys and group summaries written)
+  kRecPartial = 2,   // a speculative or repair partial of the unit is written, or skipped
+  kRecFinDone = 3,   // the unit's finisher is done; argument: kBig - expected partials
+  kRecEmaDone = 4,   // a predictor update is done
+  kRecCombDone = 5,  // a merge is done
+  kRecExit = 6,      // the writer has stopped
+};
+constexpr int kRecRing = 64;   // records per ring
+constexpr int kFinBox = 32;    // FINISH mailbox entries
 
-// A unit's partial (or the finisher's adjustment `add`) is complete; the one whose add
-// completes the count queues the unit's merges.  The add is a release (this thread's
-// partial, and what its group wrote before the group barrier, precede it); the thread
-// that completes the count takes an acquire fence before queueing, so every partial
-// counted before is visible to the merges.  A consumer issues the add and looks at the
-// result later (PendingCount), so the round trip overlaps other work.
-struct PendingCount {
-  unsigned old;
-  unsigned add;
-  int u;  // -1: none
+struct BookSmem {
+  unsigned long long rec[3][kRecRing];
+  unsigned tail[3];    // written by each ring's writer (release)
+  unsigned head[3];    // written by the bookkeeper once the records are read
+  unsigned fin[kFinBox];
+  unsigned fin_tail;   // written by the bookkeeper (release)
+  unsigned fin_head;   // written by the producer
 };
 
-__device__ inline void resolve_count(const Params& p, const FusedCtl& C, PendingCount& pc) {
-  if (pc.u < 0) return;
-  if (pc.old + pc.add == kBig) {
-    fence_acq_rel_gpu();
-    unsigned long long t[8];
-    for (int h = 0; h < p.G; ++h) t[h] = make_task(kItemCombine, pc.u, h, 0);
-    rq_push(p, C, t, p.G);
+__device__ __forceinline__ unsigned long long make_rec(unsigned op, int u, unsigned arg) {
+  return (static_cast<unsigned long long>(op) << 56) | (static_cast<unsigned long long>(u & 0xFFFFFF) << 32) | arg;
+}
+
+__device__ __forceinline__ void st_release_cta(unsigned* a, unsigned v) {
+  asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"(smem_addr(a)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_cta(const unsigned* a) {
+  unsigned v;
+  asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(a)) : "memory");
+  return v;
+}
+
+// One thread (the ring's only writer): append a record.  What the writer's group wrote
+// before its last group barrier is ordered before the record (release at CTA scope);
+// the bookkeeper's fence then publishes it at GPU scope.  Bounded wait for room.
+__device__ inline bool post_record(BookSmem* bk, int ring, unsigned& tail, unsigned long long rec, int* status) {
+  if (tail - ld_acquire_cta(&bk->head[ring]) >= static_cast<unsigned>(kRecRing)) {
+    const uint64_t t0 = global_ns();
+    while (tail - ld_acquire_cta(&bk->head[ring]) >= static_cast<unsigned>(kRecRing)) {
+      if (global_ns() - t0 > kWaitLimitNs) {
+        report(status, kDevWaitTimeout);
+        return false;
+      }
+      __nanosleep(64);
+    }
   }
-  pc.u = -1;
-}
-
-__device__ inline PendingCount issue_count(const FusedCtl& C, int u, unsigned add) {
-  return PendingCount{atom_add_release(C.done + u, add), add, u};
-}
-
-__device__ inline void count_partial(const Params& p, const FusedCtl& C, int u, unsigned add) {
-  PendingCount pc = issue_count(C, u, add);
-  resolve_count(p, C, pc);
+  bk->rec[ring][tail % kRecRing] = rec;
+  st_release_cta(&bk->tail[ring], ++tail);
+  return true;
 }
 
 // ---------------------------------------------------------------- consumer items
@@ -237,42 +262,33 @@ __device__ void sel_scores(const Params& p, const ItemDesc& it, unsigned char* r
   }
 }
 
-// The unit's selection is complete: top-K, missed set, keep mask; queue its repairs
-// and its predictor update; settle the expected partial count.  The finisher leaves
+// FINISH: the unit's selection is complete (every chunk's keys are visible): top-K,
+// missed set, keep mask; queue its repairs.  Returns the partial-count adjustment for
+// the bookkeeper (kBig - active predicted slots - missed blocks).  The finisher leaves
 // the missed blocks (+1) in the first K words of `scratch`, which it does not use
 // otherwise, so queueing them needs no global round trip.
-__device__ void finish_unit(const Params& p, const FusedCtl& C, int u, int n, unsigned char* scratch,
-                            const Grp& grp) {
+__device__ unsigned finish_unit(const Params& p, const FusedCtl& C, int u, int n, unsigned char* scratch,
+                                const Grp& grp) {
   const int nb = (n + p.bs - 1) / p.bs;
   unsigned* mlist = reinterpret_cast<unsigned*>(scratch);
   const FinishOut f = select_finish(p, u, nb, scratch, grp, C.keepf + static_cast<size_t>(u) * p.P, mlist);
-  gsync(grp);  // the unit's outputs precede the tasks that read them
+  gsync(grp);  // mlist is complete
   const int tid = grp.tid;
-  if (tid < 32) {  // one warp queues the repairs (lane-parallel) and the predictor update
-    const int nm = min(max(f.n_missed, 0), p.K);
+  const int nm = min(max(f.n_missed, 0), p.K);
+  if (tid < 32 && nm > 0) {  // one warp queues the repairs, lane-parallel; a repair reads only its word
     unsigned pos = 0;
-    if (tid == 0) pos = atomicAdd(C.words + kCtlRqTail, static_cast<unsigned>(nm + 1));
+    if (tid == 0) pos = atomicAdd(C.words + kCtlRqTail, static_cast<unsigned>(nm));
     pos = __shfl_sync(kFull, pos, 0);
-    for (int i = tid; i <= nm; i += 32) {
-      // a repair reads only its task word; the predictor update reads S_t (release)
-      const unsigned long long t = i < nm ? make_task(kItemRepair, u, i, static_cast<int>(mlist[i]) - 1)
-                                          : make_task(kItemEma, u, 0, 0);
+    for (int i = tid; i < nm; i += 32) {
       if (pos + i < static_cast<unsigned>(p.rq_cap)) {
-        if (i < nm) {
-          st_relaxed64(C.rq + pos + i, t);
-        } else {
-          st_release64(C.rq + pos + i, t);
-        }
+        st_relaxed64(C.rq + pos + i, make_task(kItemRepair, u, i, static_cast<int>(mlist[i]) - 1));
       } else {
-        report(p.status, kDevWaitTimeout);
+        report(p.status, kDevWaitTimeout);  // cannot happen: the queue holds every task of a step
         atomicExch(C.words + kCtlAbort, 1u);
       }
     }
-    __syncwarp();
-    PRR_PHASE(0, u, 6);
-    if (tid == 0) count_partial(p, C, u, kBig - static_cast<unsigned>(f.p_active + nm));
-    PRR_PHASE(0, u, 7);
   }
+  return kBig - static_cast<unsigned>(f.p_active + nm);
 }
 
 // ---------------------------------------------------------------- shared memory
@@ -285,6 +301,7 @@ struct FusedSmem {
   uint64_t* empty;       // [fslots] the consumer group is done with the slot
   int* claim;            // [1] next slot sequence number a consumer group takes
   int* bcast;            // [2][8] per-group broadcast words
+  BookSmem* bk;          // records for the bookkeeper, FINISH mailbox
 };
 
 template <int D>
@@ -304,12 +321,13 @@ __device__ __forceinline__ FusedSmem fused_smem(const Params& p, unsigned char* 
   s.empty = bars + 2 * p.fslots;
   s.claim = reinterpret_cast<int*>(bars + 3 * p.fslots);
   s.bcast = s.claim + 4;
+  s.bk = reinterpret_cast<BookSmem*>(s.bcast + 16);
   return s;
 }
 
 __host__ __device__ inline size_t fused_smem_total(int slots, int slot_bytes, size_t group_coef) {
   return 1024 + static_cast<size_t>(slots) * (slot_bytes + kAuxBytes) + 2 * group_coef +
-         3 * 8 * static_cast<size_t>(slots) + 4 * 4 + 16 * 4;
+         3 * 8 * static_cast<size_t>(slots) + 4 * 4 + 16 * 4 + sizeof(BookSmem);
 }
 
 // ---------------------------------------------------------------- producer
@@ -323,17 +341,14 @@ __device__ bool prod_emit(const Params& p, const FusedSmem& S, const CUtensorMap
   if (use > 0 && !mbar_wait_idle(&S.empty[s], (use - 1) & 1u, p.status)) return false;
   unsigned char* slot = S.slots + static_cast<size_t>(s) * p.fslot_bytes;
   unsigned char* aux = S.aux + static_cast<size_t>(s) * kAuxBytes;
-#ifdef PRR_PHASE_DEBUG
   {
     ItemDesc d = it;
-    const unsigned long long now = global_ns();
-    d.pad[0] = static_cast<int>(now & 0xFFFFFFFFu);
-    d.pad[1] = static_cast<int>(now >> 32);
+    d.seq = seq;
+#ifdef PRR_PHASE_DEBUG
+    d.t_issue = global_ns();
+#endif
     *reinterpret_cast<ItemDesc*>(aux + kAuxDesc) = d;
   }
-#else
-  *reinterpret_cast<ItemDesc*>(aux + kAuxDesc) = it;
-#endif
   const uint32_t qbytes = static_cast<uint32_t>(p.G) * D * 2;
   const uint16_t* qsrc = p.q + static_cast<size_t>(it.u) * p.G * D;
   fence_proxy_async();  // the consumers' generic writes to this slot precede the new copies
@@ -370,9 +385,10 @@ __device__ bool prod_emit(const Params& p, const FusedSmem& S, const CUtensorMap
 __device__ __forceinline__ bool warp_flag(bool v) { return __shfl_sync(kFull, v ? 1 : 0, 0) != 0; }
 
 // Producer warp.  Lane 0 drives; lanes resolve a claimed batch of main tickets in
-// parallel (one round trip for all of them).  Ready tasks come first: lane 0 always
-// holds one claimed queue index and checks it (one load, no waiting) before each
-// batch; the next batch's tickets are claimed one batch ahead.
+// parallel (one round trip for all of them).  Each pass looks first at this CTA's
+// FINISH mailbox, then at the one claimed ready-queue index lane 0 always holds (one
+// load, no waiting), then emits the batch in hand; the next batch's tickets are claimed
+// one batch ahead.
 template <int D, int BS>
 __device__ void producer(const Params& p, const FusedCtl& C, const FusedSmem& S, const CUtensorMap* kmap,
                          const CUtensorMap* vmap) {
@@ -383,6 +399,8 @@ __device__ void producer(const Params& p, const FusedCtl& C, const FusedSmem& S,
   const unsigned n_main = n_sel + static_cast<unsigned>(U) * p.P;
   const unsigned B = static_cast<unsigned>(p.fbatch);
   uint32_t seq = 0;
+  unsigned rec_tail = 0;  // lane 0: records posted to the bookkeeper
+  unsigned fin_head = 0;  // lane 0: FINISH mailbox entries taken
   bool ok = true, exhausted = false;
   // failure-detection tests set the word after the status word: selection never runs
   const bool skip_sel = p.status != nullptr && p.status[1] != 0;
@@ -394,6 +412,22 @@ __device__ void producer(const Params& p, const FusedCtl& C, const FusedSmem& S,
   uint64_t idle_t0 = 0;
 
   for (;;) {
+    // ---- a unit whose selection this CTA completed: its finisher first (critical path)
+    bool fin_emitted = false;
+    if (lane == 0 && fin_head != ld_acquire_cta(&S.bk->fin_tail)) {
+      ItemDesc it{};
+      it.kind = kItemFinish;
+      it.u = static_cast<int>(S.bk->fin[fin_head % kFinBox]);
+      it.n = checked_len(p, it.u / p.upb, solo);
+      it.trace = static_cast<int>(n_main + p.rq_cap + it.u);
+      st_release_cta(&S.bk->fin_head, ++fin_head);
+      ok = prod_emit<D, BS>(p, S, kmap, vmap, seq, it);
+      fin_emitted = true;
+    }
+    ok = warp_flag(ok);
+    if (!ok) break;
+    fin_emitted = warp_flag(fin_emitted);
+
     // One round trip per pass: lane 0 loads its claimed queue word and the abort flag
     // while the lanes load the metadata of the batch in hand; all of it is looked at
     // afterwards.
@@ -448,30 +482,8 @@ __device__ void producer(const Params& p, const FusedCtl& C, const FusedSmem& S,
       ok = false;
       break;
     }
-    // Start the batch's tiles towards L2 now: the ring takes them a few items later, and
-    // by then their copies into shared memory come from L2, so a slot's wait for its
-    // data -- and the time the ring spends not streaming -- is short.
-    if (static_cast<unsigned>(lane) < cnt && emit) {
-      if (mine.kind == kItemSel) {
-        const int c0 = mine.idx * p.fchunk_blocks;
-        const int rows = max(0, min(p.fchunk_blocks, p.maxnb - c0));
-        if (rows > 0)
-          prefetch_l2(p.summ + (static_cast<size_t>(mine.u / p.kv_div) * p.maxnb + c0) * 2 * D,
-                      static_cast<uint32_t>(rows) * 4 * D);
-      } else {
-        int tok0;
-        const int slice = kv_tile(p, mine.u / p.kv_div, mine.blk, &tok0);
-        if (!p.table || slice < p.pages * p.Hkv) {  // (a bad block-table entry is not prefetched)
-#pragma unroll
-          for (int r = 0; r < D / 64; ++r) {
-            prefetch_l2_tile_3d(kmap, r * 64, tok0, slice);
-            prefetch_l2_tile_3d(vmap, r * 64, tok0, slice);
-          }
-        }
-      }
-    }
 
-    // ---- the claimed queue entry first (repairs and merges are on the critical path)
+    // ---- the claimed queue entry (repairs and merges are on the critical path)
     const bool have_task = __shfl_sync(kFull, tq != 0ull ? 1 : 0, 0) != 0;
     if (have_task) {
       if (lane == 0) {
@@ -488,7 +500,6 @@ __device__ void producer(const Params& p, const FusedCtl& C, const FusedSmem& S,
       }
       ok = warp_flag(ok);
       if (!ok) break;
-      idle_t0 = 0;
     }
 
     // ---- the batch of main tickets
@@ -507,14 +518,14 @@ __device__ void producer(const Params& p, const FusedCtl& C, const FusedSmem& S,
           ok = prod_emit<D, BS>(p, S, kmap, vmap, seq, it);
         } else if (sd) {
           bump(p.stats, kStatSpecSkipped);
-          count_partial(p, C, it.u, 1u);
+          ok = post_record(S.bk, 2, rec_tail, make_rec(kRecPartial, it.u, 1u), p.status);
         }
       }
       ok = warp_flag(ok);
       if (!ok) break;
     }
     if (!ok) break;
-    if (cnt > 0 || have_task) {
+    if (cnt > 0 || have_task || fin_emitted) {
       idle_t0 = 0;
       continue;
     }
@@ -565,49 +576,73 @@ __device__ void producer(const Params& p, const FusedCtl& C, const FusedSmem& S,
       mbar_wait(&S.fullK[s], ph, p.status);
       mbar_wait(&S.fullV[s], ph, p.status);
     }
+    post_record(S.bk, 2, rec_tail, make_rec(kRecExit, 0, 0u), p.status);
   }
   __syncwarp();
 }
 
+// One thread: bounded wait until the slot descriptor's sequence number is `k`.
+__device__ bool wait_seq(const unsigned* seq, uint32_t k, int* status) {
+  const volatile unsigned* v = seq;
+  if (*v == k) return true;
+  const uint64_t t0 = global_ns();
+  for (int spin = 0; *v != k; ++spin) {
+    if (spin > 4) __nanosleep(64);
+    if (global_ns() - t0 > kWaitLimitNs) {
+      report(status, kDevWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- consumer groups
 // A group takes the next slot in sequence, runs its item and hands the slot back as
-// soon as it no longer reads it; the counts that other CTAs wait for come after that,
-// so the producer can refill the slot meanwhile.
+// soon as it no longer reads it; what other CTAs wait for goes to the bookkeeper as a
+// record, so the group never waits for its own global writes to complete.
 template <int D, int BS>
 __device__ void consumer(const Params& p, const FusedCtl& C, const FusedSmem& S, int group) {
   const Grp grp{static_cast<int>(threadIdx.x) - 128 * group, 128, 1 + group};
   const int tid = grp.tid;
   int* bc = S.bcast + 8 * group;
-  PendingCount pc{0u, 0u, -1};  // thread 0: the last partial's count, issued but not yet looked at
+  unsigned rec_tail = 0;  // thread 0: records posted
+  bool posted_ok = true;  // thread 0: every post went through
   for (;;) {
-    if (tid == 0) bc[0] = atomicAdd(S.claim, 1);
-    gsync(grp);
+    bool filled = true;
+    if (tid == 0) {
+      const uint32_t kc = static_cast<uint32_t>(atomicAdd(S.claim, 1));
+      bc[0] = static_cast<int>(kc);
+      // The slot's barriers are waited on by parity, which tells apart only two
+      // consecutive uses: the other group may still hold the slot's previous use (this
+      // group can run a whole ring ahead of it), so first wait until the producer has
+      // filled THIS use, which it does only once the previous one is handed back.
+      const ItemDesc* d = reinterpret_cast<const ItemDesc*>(S.aux + static_cast<size_t>(kc % p.fslots) * kAuxBytes +
+                                                            kAuxDesc);
+      filled = wait_seq(&d->seq, kc, p.status);
+    }
+    const bool filled_all = gsync_and(grp, filled);
     const uint32_t k = static_cast<uint32_t>(bc[0]);
     const int s = k % p.fslots;
     const uint32_t ph = (k / p.fslots) & 1u;
     unsigned char* slot = S.slots + static_cast<size_t>(s) * p.fslot_bytes;
     unsigned char* aux = S.aux + static_cast<size_t>(s) * kAuxBytes;
-    // before waiting for the next item, settle the last count (it may queue the merges
-    // that the next item, or the end of the step, is waiting for)
-    if (tid == 0 && pc.u >= 0 && !mbar_try_wait(&S.fullK[s], ph)) resolve_count(p, C, pc);
-    if (!gsync_and(grp, mbar_wait_idle(&S.fullK[s], ph, p.status))) {
+    if (!filled_all || !gsync_and(grp, mbar_wait_idle(&S.fullK[s], ph, p.status))) {
       if (tid == 0) {
-        resolve_count(p, C, pc);
         atomicExch(C.words + kCtlAbort, 1u);
+        post_record(S.bk, group, rec_tail, make_rec(kRecExit, 0, 0u), p.status);
       }
       return;  // the producer waits for this slot's copies before the CTA exits
     }
     const ItemDesc it = *reinterpret_cast<const ItemDesc*>(aux + kAuxDesc);
     if (it.kind == kItemExit) {
-      if (tid == 0) resolve_count(p, C, pc);
+      if (tid == 0) post_record(S.bk, group, rec_tail, make_rec(kRecExit, 0, 0u), p.status);
       return;
     }
 #ifdef PRR_PHASE_DEBUG
     unsigned long long* dbg_item =
         (it.trace >= 0 && it.trace < (1 << 16)) ? g_item[it.trace] : nullptr;
     if (dbg_item && tid == 0) {
-      dbg_item[0] = (static_cast<unsigned long long>(static_cast<unsigned>(it.pad[1])) << 32) |
-                    static_cast<unsigned>(it.pad[0]);
+      dbg_item[0] = it.t_issue;
       dbg_item[1] = global_ns();
     }
 #else
@@ -622,22 +657,14 @@ __device__ void consumer(const Params& p, const FusedCtl& C, const FusedSmem& S,
       tr[3] = static_cast<unsigned long long>(it.kind);
     }
     bool ok = true;
-    bool released = false;  // (every thread) the slot was handed back early
+    bool released = false;                 // (every thread) the slot was handed back early
+    unsigned long long rec = 0ull;         // thread 0: the record this item ends with
     if (it.kind == kItemSel) {
       sel_scores<D>(p, it, slot, aux, S.coef + group * (group_coef_bytes<D>(p) / 16), grp);
-      gsync(grp);
-      if (tid == 0) {  // this chunk's keys precede its count; the last chunk sees all keys
-        resolve_count(p, C, pc);
-        const unsigned old = atom_add_acq_rel(C.sel_cnt + it.u, 1u);
-        bc[1] = old == static_cast<unsigned>(p.fchunks - 1) ? 1 : 0;
-      }
-      gsync(grp);
-      if (bc[1]) {
-        const uint64_t t_fin = p.trace ? global_ns() : 0;
-        finish_unit(p, C, it.u, it.n, slot, grp);  // the slot is the finisher's scratch
-        if (p.trace && tid == 0)  // the finisher's own duration (ns) in the kind word's high half
-          p.trace[4 * static_cast<size_t>(it.trace) + 3] |= (global_ns() - t_fin) << 32;
-      }
+      rec = make_rec(kRecSelDone, it.u, 0u);
+    } else if (it.kind == kItemFinish) {
+      const unsigned adj = finish_unit(p, C, it.u, it.n, slot, grp);  // the slot is the finisher's scratch
+      rec = make_rec(kRecFinDone, it.u, adj);
     } else if (it.kind == kItemSpec || it.kind == kItemRepair) {
       using L = AttnTile<D, BS>;
       const bool spec = it.kind == kItemSpec;
@@ -669,52 +696,146 @@ __device__ void consumer(const Params& p, const FusedCtl& C, const FusedSmem& S,
         }
         write_empty_partial(dst, p.G, D, grp);
       }
-      if (ok) {
-        if (!released) {  // (the out-of-range path did not hand the slot back yet)
-          fence_proxy_async();
-          gsync(grp);
-          released = true;
-          if (tid == 0) mbar_arrive(&S.empty[s]);
-        }
-        gsync(grp);  // every thread's partial precedes the count
-        if (tid == 0) {
-          bump(p.stats, spec ? kStatSpecAttended : kStatRepaired);
-          resolve_count(p, C, pc);         // the previous item's count has long returned
-          pc = issue_count(C, it.u, 1u);   // looked at before the next wait or item end
-        }
-      }
+      if (tid == 0 && ok) bump(p.stats, spec ? kStatSpecAttended : kStatRepaired);
+      rec = make_rec(kRecPartial, it.u, 1u);
     } else if (it.kind == kItemEma) {
       ema_unit(p, it.u, slot, [] { return true; }, grp);
-      fence_proxy_async();
-      gsync(grp);
-      released = true;
-      if (tid == 0) {
-        mbar_arrive(&S.empty[s]);
-        resolve_count(p, C, pc);
-        red_release_add(C.words + kCtlEmaDone, 1u);
-      }
+      rec = make_rec(kRecEmaDone, it.u, 0u);
     } else if (it.kind == kItemCombine) {
       combine_head<D>(p, it.u, it.idx, slot, [] { return true; }, grp);
-      fence_proxy_async();
-      gsync(grp);
-      released = true;
-      if (tid == 0) {
-        mbar_arrive(&S.empty[s]);
-        resolve_count(p, C, pc);
-        red_release_add(C.words + kCtlCombined, 1u);
-      }
+      rec = make_rec(kRecCombDone, it.u, 0u);
     }
     if (!released) fence_proxy_async();  // generic writes to the slot precede the copies that refill it
+    // every thread's outputs (and reads of the slot) precede the slot's release and the record
     if (!gsync_and(grp, ok)) {
       if (tid == 0) {
-        resolve_count(p, C, pc);
         atomicExch(C.words + kCtlAbort, 1u);
+        post_record(S.bk, group, rec_tail, make_rec(kRecExit, 0, 0u), p.status);
       }
       return;
     }
     if (tid == 0) {
-      if (p.trace) p.trace[4 * static_cast<size_t>(it.trace) + 1] = global_ns();
       if (!released) mbar_arrive(&S.empty[s]);
+      if (rec != 0ull && posted_ok) {
+        posted_ok = post_record(S.bk, group, rec_tail, rec, p.status);
+        if (!posted_ok) atomicExch(C.words + kCtlAbort, 1u);
+      }
+      if (p.trace) p.trace[4 * static_cast<size_t>(it.trace) + 1] = global_ns();
+    }
+  }
+}
+
+// ---------------------------------------------------------------- bookkeeper
+// One warp.  Takes up to 32 records per round (one per lane) from the three rings,
+// publishes them with one release fence, applies them (one atomic per lane) and
+// queues the follow-up work of the counts that completed, after one acquire fence.
+// Ends once all three writers have posted their exit record.
+__device__ void bookkeeper(const Params& p, const FusedCtl& C, const FusedSmem& S) {
+  const int lane = threadIdx.x & 31;
+  BookSmem* bk = S.bk;
+  unsigned hd[3] = {0u, 0u, 0u};  // records taken, per ring (every lane keeps the same copy)
+  unsigned fin_tail = 0u;         // FINISH entries posted (lane 0)
+  int exits = 0;
+  uint64_t idle_t0 = global_ns();
+  for (;;) {
+    unsigned tl[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) tl[r] = __shfl_sync(kFull, lane == 0 ? ld_acquire_cta(&bk->tail[r]) : 0u, 0);
+    // this round's records: ring 0 first, then 1, then 2, at most 32 in all
+    int take[3], total = 0;
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      take[r] = min(static_cast<int>(tl[r] - hd[r]), 32 - total);
+      total += take[r];
+    }
+    if (total == 0) {
+      if (exits >= 3) break;
+      if (global_ns() - idle_t0 > kWaitLimitNs) {  // a writer never finished
+        if (lane == 0) {
+          report(p.status, kDevWaitTimeout);
+          atomicExch(C.words + kCtlAbort, 1u);
+        }
+        break;
+      }
+      __nanosleep(32);
+      continue;
+    }
+    idle_t0 = global_ns();
+    unsigned long long rec = 0ull;
+    {
+      int r = 0, i = lane;
+      while (r < 3 && i >= take[r]) i -= take[r++];
+      if (r < 3) rec = bk->rec[r][(hd[r] + i) % kRecRing];
+    }
+#pragma unroll
+    for (int r = 0; r < 3; ++r) hd[r] += take[r];
+    __syncwarp();
+    if (lane < 3) st_release_cta(&bk->head[lane], lane == 0 ? hd[0] : (lane == 1 ? hd[1] : hd[2]));
+    const unsigned op = static_cast<unsigned>(rec >> 56);
+    const int u = static_cast<int>((rec >> 32) & 0xFFFFFF);
+    const unsigned arg = static_cast<unsigned>(rec);
+    exits += __popc(__ballot_sync(kFull, op == kRecExit));
+    if (!__any_sync(kFull, op != 0u && op != kRecExit)) continue;
+
+    fence_acq_rel_gpu();  // release: every record's writes (ordered before it at CTA scope)
+    bool fin = false, comb = false, ema = false;
+    if (op == kRecSelDone) {
+      fin = atomicAdd(C.sel_cnt + u, 1u) == static_cast<unsigned>(p.fchunks - 1);
+    } else if (op == kRecPartial || op == kRecFinDone) {
+      comb = atomicAdd(C.done + u, arg) + arg == kBig;
+      ema = op == kRecFinDone;
+    } else if (op == kRecEmaDone) {
+      atomicAdd(C.words + kCtlEmaDone, 1u);
+    } else if (op == kRecCombDone) {
+      atomicAdd(C.words + kCtlCombined, 1u);
+    }
+    if (!__any_sync(kFull, fin || comb || ema)) continue;
+    fence_acq_rel_gpu();  // acquire: what the completed counts' adders published; release for the tasks
+
+    // global tasks: the unit's predictor update, its G merges
+    const int ntask = (ema ? 1 : 0) + (comb ? p.G : 0);
+    const int inc = warp_inclusive_sum(ntask);
+    const int all = __shfl_sync(kFull, inc, 31);
+    if (all > 0) {
+      unsigned pos = 0;
+      if (lane == 0) pos = atomicAdd(C.words + kCtlRqTail, static_cast<unsigned>(all));
+      pos = __shfl_sync(kFull, pos, 0) + static_cast<unsigned>(inc - ntask);
+      for (int t = 0; t < ntask; ++t, ++pos) {
+        const unsigned long long w = (ema && t == 0) ? make_task(kItemEma, u, 0, 0)
+                                                     : make_task(kItemCombine, u, t - (ema ? 1 : 0), 0);
+        if (pos < static_cast<unsigned>(p.rq_cap)) {
+          st_relaxed64(C.rq + pos, w);
+        } else {
+          report(p.status, kDevWaitTimeout);  // cannot happen: the queue holds every task of a step
+          atomicExch(C.words + kCtlAbort, 1u);
+        }
+      }
+    }
+    // FINISH of the units whose selection completed here: this CTA's mailbox, in lane order
+    if (__any_sync(kFull, fin)) {
+      unsigned m = __ballot_sync(kFull, fin);
+      while (m) {
+        const int l = __ffs(m) - 1;
+        m &= m - 1u;
+        const int fu = __shfl_sync(kFull, u, l);
+        if (lane == 0) {
+          bool room = fin_tail - ld_acquire_cta(&bk->fin_head) < static_cast<unsigned>(kFinBox);
+          if (!room) {
+            const uint64_t t0 = global_ns();
+            while (!(room = fin_tail - ld_acquire_cta(&bk->fin_head) < static_cast<unsigned>(kFinBox))) {
+              if (global_ns() - t0 > kWaitLimitNs) break;
+              __nanosleep(64);
+            }
+          }
+          if (room) {
+            bk->fin[fin_tail % kFinBox] = static_cast<unsigned>(fu);
+            st_release_cta(&bk->fin_tail, ++fin_tail);
+          } else {
+            report(p.status, kDevWaitTimeout);
+            atomicExch(C.words + kCtlAbort, 1u);
+          }
+        }
+      }
     }
   }
 }
@@ -735,6 +856,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     unsigned* other = p.ctl + static_cast<size_t>(1 - p.parity) * p.ctl_words;
     for (int i = tid; i < p.ctl_words; i += blockDim.x) other[i] = 0u;
   }
+  if (tid < 3) {
+    S.bk->tail[tid] = 0u;
+    S.bk->head[tid] = 0u;
+  }
   if (tid == 0) {
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
@@ -742,14 +867,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       mbar_init(&S.fullK[i], 1);
       mbar_init(&S.fullV[i], 1);
       mbar_init(&S.empty[i], 1);
+      reinterpret_cast<ItemDesc*>(S.aux + static_cast<size_t>(i) * kAuxBytes + kAuxDesc)->seq = kNoSeq;
     }
     S.claim[0] = 0;
+    S.bk->fin_tail = 0u;
+    S.bk->fin_head = 0u;
     fence_barrier_init();
   }
   __syncthreads();
   const int warp = tid >> 5;
   if (warp == kProducerWarp) {
     producer<D, BS>(p, C, S, &kmap, &vmap);
+  } else if (warp == kBookWarp) {
+    bookkeeper(p, C, S);
   } else {
     consumer<D, BS>(p, C, S, warp / 4);
   }
@@ -761,7 +891,7 @@ void fused_geometry(Params& p, int sms) {
   p.fchunks = (p.maxnb + p.fchunk_blocks - 1) / p.fchunk_blocks;
   const long long n_main = static_cast<long long>(p.units) * (p.fchunks + p.P);
   const long long b = n_main / (4LL * sms);
-  p.fbatch = static_cast<int>(b < 1 ? 1 : (b > 8 ? 8 : b));
+  p.fbatch = static_cast<int>(b < 1 ? 1 : (b > 4 ? 4 : b));
   p.rq_cap = p.units * (1 + p.K + p.G);
   p.ctl_words = static_cast<int>(fused_ctl_words(p.units, p.P, p.K, p.G));
 }
@@ -769,7 +899,8 @@ void fused_geometry(Params& p, int sms) {
 template <int D, int BS>
 static size_t fused_smem_for(Params& p) {
   p.fslot_bytes = static_cast<int>(fused_slot_bytes<D, BS>(p));
-  const long long room = 227LL * 1024 - 1024 - 128 - 2 * static_cast<long long>(group_coef_bytes<D>(p));
+  const long long room = 227LL * 1024 - 1024 - 128 - static_cast<long long>(sizeof(BookSmem)) -
+                         2 * static_cast<long long>(group_coef_bytes<D>(p));
   const long long slots = room / (p.fslot_bytes + kAuxBytes + 24);
   p.fslots = static_cast<int>(slots < 8 ? (slots < 0 ? 0 : slots) : 8);
   return fused_smem_total(p.fslots, p.fslot_bytes, group_coef_bytes<D>(p));

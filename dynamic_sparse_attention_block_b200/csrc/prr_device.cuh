@@ -197,6 +197,11 @@ __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Shared-memory add without a return value (the issuing thread does not wait for it).
+__device__ __forceinline__ void red_shared_add(unsigned* a, unsigned v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_addr(a)), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -256,14 +261,6 @@ __device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
 // Hint: start bringing `bytes` (multiple of 16, 16-byte aligned) of global memory into L2.
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// Hint: start bringing a 3-D tile of a tensor map into L2 (no shared memory, no barrier).
-__device__ __forceinline__ void prefetch_l2_tile_3d(const CUtensorMap* map, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

@@ -85,27 +85,29 @@ __device__ __forceinline__ void load_group_coef(const Params& p, const uint16_t*
 }
 
 // Bound of one block from its summary row in shared memory.  Lanes start at rotated
-// chunks, so 32 lanes reading 32 consecutive rows hit distinct banks.
+// chunks, so 32 lanes reading 32 consecutive rows hit distinct banks.  Four
+// independent accumulators (one per pair of products of a chunk) keep four fused
+// multiply-add chains in flight instead of one; exact on the dyadic grid in any order.
 template <int D>
 __device__ __forceinline__ float score_summary_row(const unsigned char* row, const float4* lo4,
                                                    const float4* hi4, int lane) {
   constexpr int C = 4 * D / 16;  // 16-byte chunks per row
-  float acc = 0.f;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 8
   for (int i = 0; i < C; ++i) {
     const int cc = (i + lane) & (C - 1);
     const uint4 w = *reinterpret_cast<const uint4*>(row + cc * 16);
     const float4 a = lo4[cc], z = hi4[cc];
-    acc = fmaf(a.x, bf16_lo(w.x), acc);
-    acc = fmaf(a.y, bf16_hi(w.x), acc);
-    acc = fmaf(a.z, bf16_lo(w.y), acc);
-    acc = fmaf(a.w, bf16_hi(w.y), acc);
-    acc = fmaf(z.x, bf16_lo(w.z), acc);
-    acc = fmaf(z.y, bf16_hi(w.z), acc);
-    acc = fmaf(z.z, bf16_lo(w.w), acc);
-    acc = fmaf(z.w, bf16_hi(w.w), acc);
+    a0 = fmaf(a.x, bf16_lo(w.x), a0);
+    a1 = fmaf(a.z, bf16_lo(w.y), a1);
+    a2 = fmaf(z.x, bf16_lo(w.z), a2);
+    a3 = fmaf(z.z, bf16_lo(w.w), a3);
+    a0 = fmaf(a.y, bf16_hi(w.x), a0);
+    a1 = fmaf(a.w, bf16_hi(w.y), a1);
+    a2 = fmaf(z.y, bf16_hi(w.z), a2);
+    a3 = fmaf(z.w, bf16_hi(w.w), a3);
   }
-  return acc;
+  return (a0 + a1) + (a2 + a3);
 }
 
 // Selector variant (group max): the block score is the LARGEST of the group's per-head
@@ -342,7 +344,6 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
     }
   }
   PRR_PHASE(0, u, 2);
-  PRR_PHASE(0, u, 3);
   if (tie_masks) {
     // the first K_eff tied blocks in index order: trim the maximal groups' masks
     if (warp == 0) {
@@ -386,6 +387,7 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
         },
         bm_sel, bm_eq, grp);
   }
+  PRR_PHASE(0, u, 3);
   // three warps in parallel: selected list, missed list, keep mask
   int nm = 0;
   if (warp == 0) {
@@ -418,12 +420,12 @@ __device__ inline FinishOut select_finish(const Params& p, int u, int nb, unsign
     p.keep[static_cast<size_t>(u) * p.P + j] = static_cast<uint8_t>(kv);
     if (keepf) keepf[j] = 1u | (kv << 1);
   }
+  PRR_PHASE(0, u, 4);
   // active predicted slots (CTA sum of the per-thread counts)
   if (tid == 0) misc[3] = 0;
   gsync(grp);
   if (active_local) atomicAdd(&misc[3], active_local);
   gsync(grp);
-  PRR_PHASE(0, u, 4);
   PRR_PHASE(0, u, 5);
   const int path = take_all ? kStatTakeAll : (tie_masks ? kStatTieMasks : kStatKeySearch);
   if (tid == 0 && keff > 0) bump(p.stats, path);

@@ -4,10 +4,9 @@
 // Ranking order everywhere: larger key first, ties broken by the lower index.  The
 // top-k set is therefore {key > T} plus the lowest-index entries with key == T, where
 // T is the k-th largest key (with multiplicity).  T is found MSB-first, 8 bits per
-// pass, from a shared-memory histogram (shared atomics; the lanes of a warp that agree
-// with its first active lane add in one atomic, which keeps heavy ties cheap).  Sets are then held as bitmaps (one ballot per
-// 32 entries); trimming the ties and writing a set in ascending index order take one
-// warp, popcounts and a shuffle prefix sum.  These routines run once per step on the
+// pass, from a shared-memory histogram (one shared-memory reduction per key).  Sets
+// are then held as bitmaps (one ballot per 32 entries); trimming the ties and writing
+// a set in ascending index order take one warp, popcounts and a shuffle prefix sum.  These routines run once per step on the
 // critical path, so they use few barriers and no CTA-wide scans.  Every thread of the
 // group must call the functions that synchronise it (marked "Group"; see Grp).
 #pragma once
@@ -40,12 +39,17 @@ template <typename KeyFn, typename MemberFn>
 __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, unsigned* hist, int* bc,
                                       int* n_gt, const Grp& grp) {
   const int tid = grp.tid, lane = tid & 31, warp = tid >> 5, NT = grp.nt, nw = NT >> 5;
+  constexpr int U = 4;  // keys per thread per round: independent loads in flight
   unsigned kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int i = tid; i < n; i += NT) {
-    if (member(i)) {
-      const uint32_t v = key(i);
-      kmin = min(kmin, v);
-      kmax = max(kmax, v);
+  for (int base = 0; base < n; base += U * NT) {
+#pragma unroll
+    for (int q = 0; q < U; ++q) {
+      const int i = base + q * NT + tid;
+      if (i < n && member(i)) {
+        const uint32_t v = key(i);
+        kmin = min(kmin, v);
+        kmax = max(kmax, v);
+      }
     }
   }
   kmin = __reduce_min_sync(kFull, kmin);
@@ -73,25 +77,25 @@ __device__ uint32_t radix_kth_largest(int n, int k, KeyFn key, MemberFn member, 
   for (int shift = 24 - 8 * skip; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += NT) hist[i] = 0u;
     gsync(grp);
-    for (int base = 0; base < n; base += NT) {  // warp-uniform trip count
-      const int i = base + tid;
-      unsigned dg = 0u;
-      bool act = false;
-      if (i < n && member(i)) {
-        const uint32_t kv = key(i);
-        act = (kv & pmask) == prefix;
-        dg = (kv >> shift) & 0xFFu;
+    for (int base = 0; base < n; base += U * NT) {  // warp-uniform trip count
+      unsigned dg[U];
+      bool act[U];
+#pragma unroll
+      for (int q = 0; q < U; ++q) {
+        const int i = base + q * NT + tid;
+        dg[q] = 0u;
+        act[q] = false;
+        if (i < n && member(i)) {
+          const uint32_t kv = key(i);
+          act[q] = (kv & pmask) == prefix;
+          dg[q] = (kv >> shift) & 0xFFu;
+        }
       }
-      // Heavily tied keys share a bin: the lanes agreeing with the first active lane
-      // add in one atomic (a per-lane atomic on one address would serialise).
-      const unsigned am = __ballot_sync(kFull, act);
-      if (am) {
-        const int leader = __ffs(am) - 1;
-        const unsigned d0 = __shfl_sync(kFull, dg, leader);
-        const unsigned same = __ballot_sync(kFull, act && dg == d0);
-        if (lane == leader) atomicAdd(&hist[d0], static_cast<unsigned>(__popc(same)));
-        else if (act && dg != d0) atomicAdd(&hist[dg], 1u);
-      }
+      // One shared-memory reduction per key (no return value, so the issuing warp does
+      // not wait for it); aggregating equal digits first costs more than it saves.
+#pragma unroll
+      for (int q = 0; q < U; ++q)
+        if (act[q]) red_shared_add(&hist[dg[q]], 1u);
     }
     gsync(grp);
     if (warp == 0) {
@@ -143,14 +147,23 @@ template <typename CmpFn>
 __device__ void select_bitmap(int n, int take_equal, CmpFn cmp, unsigned* bm, unsigned* eq, const Grp& grp) {
   const int lane = grp.tid & 31, warp = grp.tid >> 5, nw = grp.nt >> 5;
   const int W = (n + 31) / 32;
-  for (int wd = warp; wd < W; wd += nw) {
-    const int i = wd * 32 + lane;
-    const int c = i < n ? cmp(i) : -1;
-    const unsigned gt = __ballot_sync(kFull, c > 0);
-    const unsigned e = __ballot_sync(kFull, c == 0);
-    if (lane == 0) {
-      bm[wd] = gt;
-      eq[wd] = e;
+  constexpr int U = 4;  // words per warp per round: independent comparisons in flight
+  for (int w0 = warp; w0 < W; w0 += U * nw) {
+    int c[U];
+#pragma unroll
+    for (int q = 0; q < U; ++q) {
+      const int i = (w0 + q * nw) * 32 + lane;
+      c[q] = i < n ? cmp(i) : -1;
+    }
+#pragma unroll
+    for (int q = 0; q < U; ++q) {
+      const int wd = w0 + q * nw;
+      const unsigned gt = __ballot_sync(kFull, c[q] > 0);
+      const unsigned e = __ballot_sync(kFull, c[q] == 0);
+      if (lane == 0 && wd < W) {
+        bm[wd] = gt;
+        eq[wd] = e;
+      }
     }
   }
   gsync(grp);

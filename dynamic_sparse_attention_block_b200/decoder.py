@@ -129,13 +129,13 @@ class PRRDecoder:
 
     def fused_items(self, sms: Optional[int] = None) -> dict:
         """Trace records of one fused launch, in record order: the main work (selection
-        chunks, then speculative slots) and the task records (repairs, predictor
-        updates and merges, in the order they were queued)."""
+        chunks, then speculative slots), the task records (repairs, predictor updates
+        and merges, in the order they were queued) and one finisher record per unit."""
         d = self.dims
         sms = sms or torch.cuda.get_device_properties(self.device).multi_processor_count
         chunk = min(128, max(32, -(-(-(-d.units * d.maxnb // (2 * sms))) // 32) * 32))
         return {"sel": d.units * -(-d.maxnb // chunk), "spec": d.units * d.P,
-                "tasks": d.units * (1 + d.K + d.group)}
+                "tasks": d.units * (1 + d.K + d.group), "finish": d.units}
 
     def enable_trace(self, on: bool = True) -> None:
         """Record start/end times of every work item of the fused launches."""
@@ -274,14 +274,15 @@ class PRRDecoder:
         return _abi.prr_get_device_status(self.ws)
 
 
-KINDS = {1: "sel", 2: "spec", 3: "repair", 4: "ema", 5: "combine"}
+KINDS = {1: "sel", 2: "spec", 3: "repair", 4: "ema", 5: "combine", 6: "finish"}
 
 
 def summarize_trace(trace) -> dict:
     """Per item kind of one fused launch: how many items ran, when the first and last
     started and the last ended (microseconds after the earliest start), and the p50 /
-    mean / max item duration.  `trace` is the [records][4] array of prr_step_buffers
-    (start ns, end ns, SM << 32 | group << 16 | CTA, kind | finisher ns << 32)."""
+    mean / max item duration; "finisher" repeats the count and durations of the top-K
+    finisher items.  `trace` is the [records][4] array of prr_step_buffers (start ns,
+    end ns, SM << 32 | group << 16 | CTA, kind)."""
     import numpy as np
     tr = np.asarray(trace, dtype=np.int64)
     ran = tr[:, 0] > 0
@@ -290,9 +291,9 @@ def summarize_trace(trace) -> dict:
     t0 = tr[ran, 0].min()
     out = {"end_us": float((tr[ran, 1].max() - t0) / 1e3)}
     kinds = tr[:, 3] & 0xFFFFFFFF
-    fin = (tr[:, 3] >> 32) / 1e3
-    if (fin > 0).any():
-        f = fin[fin > 0]
+    fin = ran & (kinds == 6)
+    if fin.any():
+        f = (tr[fin, 1] - tr[fin, 0]) / 1e3
         out["finisher"] = {"n": int(len(f)), "dur_p50_us": float(np.median(f)), "dur_max_us": float(f.max())}
     for code, kind in KINDS.items():
         seg = tr[ran & (kinds == code)]

@@ -146,13 +146,13 @@ typedef struct {
   const uint16_t* v_new;
   /* Optional (NULL: off).  prr_decode_step_fused records, for every item its CTAs run,
    * trace[4i..4i+3] = {start ns, end ns, (SM id << 32) | (consumer group << 16) | CTA,
-   * kind | (finisher ns << 32)} (%globaltimer; kind 1 selection chunk, 2 speculative
-   * block, 3 repair block, 4 predictor update, 5 merge; a selection chunk that ran its
-   * unit's top-K records the top-K's duration in the high half).  Records: first the main work in queue order --
-   * units*ceil(maxnb/C) selection chunks (C blocks each: units*maxnb/(2*SMs) rounded up
-   * to a multiple of 32, clamped to [32, 128]), then units*P speculative slots -- then
-   * units*(1+K+G) task records in the order the tasks were queued.  Items that did not
-   * run stay zero.  Size: 4 * (units*(ceil(maxnb/C) + P) + units*(1+K+G)) words. */
+   * kind} (%globaltimer; kind 1 selection chunk, 2 speculative block, 3 repair block,
+   * 4 predictor update, 5 merge, 6 top-K finisher).  Records: first the main work in
+   * queue order -- units*ceil(maxnb/C) selection chunks (C blocks each:
+   * units*maxnb/(2*SMs) rounded up to a multiple of 32, clamped to [32, 128]), then
+   * units*P speculative slots -- then units*(1+K+G) task records in the order the tasks
+   * were queued, then one finisher record per unit.  Items that did not run stay zero.
+   * Size: 4 * (units*(ceil(maxnb/C) + P) + units*(1+K+G) + units) words. */
   unsigned long long* trace;
   /* Optional (NULL: off).  Eight counters the step adds to (atomically; the caller
    * zeroes them):  [0] units whose top-K came straight from the 32-block group tie

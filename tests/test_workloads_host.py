@@ -69,16 +69,19 @@ def test_batch_override_for_reduced_captures():
 
 def test_trace_summary_on_a_synthetic_timeline():
     """Records carry their item kind (1 selection chunk, 2 speculative block, 3 repair,
-    4 predictor, 5 merge); records that never ran stay zero and are ignored."""
+    4 predictor, 5 merge, 6 finisher); records that never ran stay zero and are
+    ignored."""
     from dynamic_sparse_attention_block_b200.decoder import summarize_trace
     ns = 1000
     trace = np.array([[10 * ns, 14 * ns, (3 << 32) | 1, 1],
                       [11 * ns, 15 * ns, (4 << 32) | 2, 1],
                       [15 * ns, 20 * ns, (3 << 32) | (1 << 16) | 1, 3],
                       [12 * ns, 16 * ns, (5 << 32) | 3, 2],
+                      [16 * ns, 19 * ns, (5 << 32) | 3, 6],
                       [0, 0, 0, 0]], np.int64)  # last record never ran
     s = summarize_trace(trace)
     assert s["sel"]["n"] == 2 and s["sel"]["start_min_us"] == 0.0 and s["sel"]["end_max_us"] == 5.0
     assert s["repair"]["dur_p50_us"] == 5.0 and s["repair"]["sms"] == 1
     assert s["spec"]["n"] == 1 and s["spec"]["start_min_us"] == 2.0
     assert s["ema"]["n"] == 0 and s["end_us"] == 10.0
+    assert s["finish"]["n"] == 1 and s["finisher"] == {"n": 1, "dur_p50_us": 3.0, "dur_max_us": 3.0}
