@@ -287,13 +287,14 @@ __device__ bool attn_compute(const Params& p, const uint16_t* q, int blk, int n,
   return true;
 }
 
-// Both steps in one group (standalone kernels): partial of block `blk` of unit u.
-// `smem` is 1024-byte aligned with AttnTile::bytes free; bars[0], bars[1] are
-// initialised mbarriers (count 1) whose current phase parity is `phase`.
+// Both steps in one group: partial of block `blk` of unit u.  `smem` is 1024-byte
+// aligned with AttnTile::bytes free; bars[0], bars[1] are initialised mbarriers (count
+// 1) whose current phase parity is `phase`.  patch_k / patch_v: see attn_compute.
 template <int D, int BS>
 __device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CUtensorMap* vmap, int u,
                               int blk, int n, const PartialDst& dst, unsigned char* smem, uint64_t* bars,
-                              uint32_t phase, const Grp& grp) {
+                              uint32_t phase, const Grp& grp, const uint16_t* patch_k = nullptr,
+                              const uint16_t* patch_v = nullptr) {
   using L = AttnTile<D, BS>;
   unsigned char* sK = smem;
   unsigned char* sV = smem + L::TILEB;
@@ -304,7 +305,7 @@ __device__ bool block_partial(const Params& p, const CUtensorMap* kmap, const CU
   }
   return attn_compute<D, BS>(p, p.q + static_cast<size_t>(u) * p.G * D, blk, n, dst, sK, sV,
                              reinterpret_cast<float*>(smem + 2 * L::TILEB), &bars[0], &bars[1], phase, grp,
-                             [] {});
+                             [] {}, patch_k, patch_v);
 }
 
 }  // namespace prr

@@ -67,10 +67,8 @@ struct Params {
   int ctl_words;     // words per copy
   int fchunks;       // SEL items per unit
   int fchunk_blocks; // blocks per SEL item (multiple of 32, at most 128)
-  int fslots;        // item slots of the shared-memory ring
-  int fslot_bytes;   // bytes of one slot's main area (tiles, summary rows or task scratch)
-  int fbatch;        // main tickets a producer claims per atomic
-  int rq_cap;        // ready-queue entries per control-word copy
+  int fregion;       // bytes of the per-CTA shared-memory union of the fused step
+  int rep_items;     // REPAIR items per unit of the fused step: item r repairs missed slots r, r + rep_items, ...
   // caller buffers (any may be null when the kernel does not use it)
   const uint16_t* q;        // [B][Hq][d] bf16
   const uint16_t* k_new;    // [B][Hkv][d] bf16 token appended by the fused step (append_kv)

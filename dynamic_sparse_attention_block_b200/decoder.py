@@ -128,14 +128,13 @@ class PRRDecoder:
         return e
 
     def fused_items(self, sms: Optional[int] = None) -> dict:
-        """Trace records of one fused launch, in record order: the main work (selection
-        chunks, then speculative slots), the task records (repairs, predictor updates
-        and merges, in the order they were queued) and one finisher record per unit."""
+        """Work items of one fused launch, in ticket (and trace record) order: selection
+        chunks, finishers, predictor updates, speculative slots, repair items and merges."""
         d = self.dims
-        sms = sms or torch.cuda.get_device_properties(self.device).multi_processor_count
-        chunk = min(128, max(32, -(-(-(-d.units * d.maxnb // (2 * sms))) // 32) * 32))
-        return {"sel": d.units * -(-d.maxnb // chunk), "spec": d.units * d.P,
-                "tasks": d.units * (1 + d.K + d.group), "finish": d.units}
+        chunk = min(128, max(32, -(-(-(-d.units * d.maxnb // 512)) // 32) * 32))
+        rep = min(d.K, max(4, -(-1024 // d.units)))
+        return {"sel": d.units * -(-d.maxnb // chunk), "finish": d.units, "ema": d.units, "spec": d.units * d.P,
+                "repair": d.units * rep, "combine": d.units * d.group}
 
     def enable_trace(self, on: bool = True) -> None:
         """Record start/end times of every work item of the fused launches."""

@@ -144,15 +144,14 @@ typedef struct {
    * inside its one launch; prr_decode_step launches the append first. */
   const uint16_t* k_new;
   const uint16_t* v_new;
-  /* Optional (NULL: off).  prr_decode_step_fused records, for every item its CTAs run,
-   * trace[4i..4i+3] = {start ns, end ns, (SM id << 32) | (consumer group << 16) | CTA,
-   * kind} (%globaltimer; kind 1 selection chunk, 2 speculative block, 3 repair block,
-   * 4 predictor update, 5 merge, 6 top-K finisher).  Records: first the main work in
-   * queue order -- units*ceil(maxnb/C) selection chunks (C blocks each:
-   * units*maxnb/(2*SMs) rounded up to a multiple of 32, clamped to [32, 128]), then
-   * units*P speculative slots -- then units*(1+K+G) task records in the order the tasks
-   * were queued, then one finisher record per unit.  Items that did not run stay zero.
-   * Size: 4 * (units*(ceil(maxnb/C) + P) + units*(1+K+G) + units) words. */
+  /* Optional (NULL: off).  prr_decode_step_fused records, for every work item its CTAs
+   * run, trace[4i..4i+3] = {start ns, end ns, (SM id << 32) | CTA, kind} (%globaltimer;
+   * kind 1 selection chunk, 6 top-K finisher, 4 predictor update, 2 speculative block,
+   * 3 repair item, 5 merge).  Records follow the items' ticket order: units*ceil(maxnb/C)
+   * selection chunks (C blocks each: units*maxnb/512 rounded up to a multiple of 32,
+   * clamped to [32, 128]), units finishers, units predictor updates, units*P speculative
+   * slots, units*R repair items (R = min(K, max(4, ceil(1024/units)))), units*G merges.
+   * Items that did not run stay zero.  Size: 4 * (that many records) words. */
   unsigned long long* trace;
   /* Optional (NULL: off).  Eight counters the step adds to (atomically; the caller
    * zeroes them):  [0] units whose top-K came straight from the 32-block group tie
