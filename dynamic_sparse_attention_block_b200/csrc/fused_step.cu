@@ -93,7 +93,7 @@ __device__ __forceinline__ FusedCtl ctl_view(const Params& p, int parity) {
 
 // CTA-wide bounded wait until *flag >= target.  Thread 0 polls; the verdict is shared,
 // and every thread gets the flag value thread 0 saw last in *seen (if given).
-__device__ bool wait_geq(const unsigned* flag, unsigned target, const FusedCtl& C, int* status, int* sh,
+static __device__ bool wait_geq(const unsigned* flag, unsigned target, const FusedCtl& C, int* status, int* sh,
                          unsigned* seen = nullptr) {
   if (threadIdx.x == 0) {
     int ok = 1;
@@ -137,7 +137,7 @@ __device__ __forceinline__ void count_done(unsigned* counter) {
 // advances seq_lens when the launch appended the step's token (every item has read
 // seq_lens by then: each reads it as it starts, and all of them start before the last
 // merge can finish).
-__device__ void count_tail(const Params& p, const FusedCtl& C) {
+static __device__ void count_tail(const Params& p, const FusedCtl& C) {
   __syncthreads();
   if (threadIdx.x == 0) {
     const unsigned total = static_cast<unsigned>(p.units) * (p.G + 1);
@@ -244,7 +244,7 @@ __device__ void sel_item(const Params& p, const FusedCtl& C, int u, int chunk, u
 }
 
 // ---------------------------------------------------------------- FIN item
-__device__ void fin_item(const Params& p, const FusedCtl& C, int u, unsigned char* smem, int* sh) {
+static __device__ void fin_item(const Params& p, const FusedCtl& C, int u, unsigned char* smem, int* sh) {
   if (!wait_geq(C.sel_cnt + u, static_cast<unsigned>(p.fchunks), C, p.status, sh)) return;
   const int n = checked_len(p, u / p.upb, cta_grp());
   const int nb = (n + p.bs - 1) / p.bs;
