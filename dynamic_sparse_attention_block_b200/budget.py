@@ -4,9 +4,12 @@ PRR (abstract) sizes its speculative work from profiling so that it stays off th
 critical path; its limitations list says the overheads at context lengths between the
 profiled ones come from polynomial regressions.  This module:
 
-- profiles, on the GPU, the selection time and the speculation time of the two-stream
-  decode step (``prr_decode_step`` with its per-kernel timing marks) over a grid of
-  context lengths and speculation budgets (``profile``);
+- profiles, on the GPU, the selection time and the speculation time over a grid of
+  context lengths and speculation budgets: of the two-stream decode step
+  (``prr_decode_step`` with its per-kernel timing marks, ``profile``) or of the fused
+  single-launch step, from the launch's per-item trace (``profile_fused``: selection
+  ends when the last top-K finisher does, speculation when the last speculative block
+  does, both measured from the launch's first item);
 - fits one polynomial in the context length to the selection times and one per
   budget to the speculation times (``SpecBudget.fit``, through ``prr_budget_fit``);
 - answers, for any context length, the largest profiled budget whose speculation is
@@ -74,6 +77,53 @@ def profile(base: _abi.Dims, contexts: Sequence[int], p_grid: Sequence[int], ste
                 if t >= warmup:
                     s_list.append(_elapsed_us(marks["t_begin"], marks["t_select_end"]))
                     p_list.append(_elapsed_us(marks["t_spec_begin"], marks["t_spec_end"]))
+            status = dec.device_status()
+            if status != 0:
+                raise RuntimeError(f"device status {status} while profiling context {n0}, P {p}")
+            sel_us[(n0, p)] = statistics.median(s_list)
+            spec_us[(n0, p)] = statistics.median(p_list)
+            del dec
+    return Profile(list(contexts), list(p_grid), sel_us, spec_us)
+
+
+def profile_fused(base: _abi.Dims, contexts: Sequence[int], p_grid: Sequence[int], steps: int = 8,
+                  warmup: int = 3, seed: int = 0) -> Profile:
+    """Time selection and speculation inside the fused step for every (context, P).
+
+    The same decoders and inputs as ``profile``; each step runs ``step_fused`` with the
+    trace on.  From the trace (microseconds after the launch's first item starts):
+    selection time = when the last selection chunk or top-K finisher ends, speculation
+    time = when the last speculative block ends.  Speculation is off the critical path
+    when it ends no later than selection."""
+    import torch
+
+    from .decoder import PRRDecoder, summarize_trace
+
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    sel_us, spec_us = {}, {}
+    for n0 in contexts:
+        for p in p_grid:
+            dims = dataclasses.replace(base, cap_tokens=n0 + warmup + steps + 1, P=p)
+            dec = PRRDecoder(dims)
+            shape = (dims.B, dims.Hkv, n0, dims.d)
+            dec.k_cache[:, :, :n0].copy_(torch.randn(shape, generator=gen, device="cuda").to(torch.bfloat16))
+            dec.v_cache[:, :, :n0].copy_(torch.randn(shape, generator=gen, device="cuda").to(torch.bfloat16))
+            dec.prefill(dec.k_cache[:, :, :n0], dec.v_cache[:, :, :n0], n0)
+            dec.enable_trace(True)
+            s_list, p_list = [], []
+            kv = (dims.B, dims.Hkv, dims.d)
+            for t in range(warmup + steps):
+                q = torch.randn((dims.B, dims.Hq, dims.d), generator=gen, device="cuda").to(torch.bfloat16)
+                kn = torch.randn(kv, generator=gen, device="cuda").to(torch.bfloat16)
+                vn = torch.randn(kv, generator=gen, device="cuda").to(torch.bfloat16)
+                dec.trace.zero_()
+                dec.step_fused(q, k_new=kn, v_new=vn)
+                torch.cuda.synchronize()
+                if t >= warmup:
+                    tr = summarize_trace(dec.trace.cpu().numpy())
+                    s_list.append(max(tr["sel"].get("end_max_us", 0.0), tr["finish"].get("end_max_us", 0.0)))
+                    p_list.append(tr["spec"].get("end_max_us", 0.0))
             status = dec.device_status()
             if status != 0:
                 raise RuntimeError(f"device status {status} while profiling context {n0}, P {p}")
