@@ -19,6 +19,10 @@
 // Selection work is handed out first, so the critical path (select -> repair -> merge)
 // starts at once and speculation streams while it runs; a dependent item waits for
 // its inputs in the CTA that took it, so a result is picked up the moment it exists.
+// After the predictor updates, each unit's REPAIR and COMBINE tickets follow its SPEC
+// tickets a fixed lag later (about two rounds of the resident grid), so the merges of
+// the early units run while the later units still stream instead of all waiting for the
+// last speculative block.
 //
 // Waits only ever target items with a smaller index, which were taken by CTAs that are
 // already running, so every wait ends without any co-residency assumption.  Each wait
@@ -257,6 +261,46 @@ static __device__ void fin_item(const Params& p, const FusedCtl& C, int u, unsig
   }
 }
 
+// Tickets after the predictor updates (t counts from the first of them), with
+// Lc = min(dep_lag, units) and M = R + G dependent items per unit: first the SPEC
+// tickets of units 0..Lc-1 (P each); then, for k = 0..units-Lc-1, the SPEC tickets of
+// unit Lc+k followed by unit k's R REPAIR and G COMBINE tickets; last the dependent
+// tickets of units units-Lc..units-1.  Every dependent ticket comes after all of its
+// unit's SPEC tickets.  Returns false for a SPEC ticket (*idx = unit * P + slot), true
+// for a dependent one (*kind 3 with *idx = unit * R + r, or 5 with *idx = unit * G + h).
+__device__ __forceinline__ bool decode_tail(const Params& p, int t, int U, int R, int* idx, int* kind) {
+  const int P = p.P, M = R + p.G;
+  const int Lc = min(p.dep_lag, U);
+  int v, r;  // unit and index of a dependent ticket
+  if (t < Lc * P) {
+    *idx = t;
+    return false;
+  }
+  t -= Lc * P;
+  const int mid = (U - Lc) * (P + M);
+  if (t < mid) {
+    const int k = t / (P + M), q = t % (P + M);
+    if (q < P) {
+      *idx = (Lc + k) * P + q;
+      return false;
+    }
+    v = k;
+    r = q - P;
+  } else {
+    t -= mid;
+    v = U - Lc + t / M;
+    r = t % M;
+  }
+  if (r < R) {
+    *kind = 3;
+    *idx = v * R + r;
+  } else {
+    *kind = 5;
+    *idx = v * p.G + (r - R);
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- the kernel
 template <int D, int BS>
 __global__ void __launch_bounds__(kFusedThreads, 3) fused_step_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -308,7 +352,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fused_step_kernel(const __gr
     if (it >= total) break;
     fence_proxy_async();  // generic shared-memory writes of the last item precede new copies
     const int item_id = it;
-    int kind = 0;
+    int kind = 0, kind_tail = 0;
     if (p.trace && tid == 0) {
       unsigned smid;
       asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
@@ -327,7 +371,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fused_step_kernel(const __gr
       kind = 4;
       ema_unit(p, it, smem, [&] { return wait_geq(C.sel_done + it, 1u, C, p.status, sh); }, cta_grp());
       count_tail(p, C);
-    } else if ((it -= n_ema) < n_spec) {  // speculation
+    } else if (!decode_tail(p, it - n_ema, U, R, &it, &kind_tail)) {  // speculation
       kind = 2;
       if (tid == 0) next_ticket = atomicAdd(C.words + kCtlWork, 1u);
       const int u = it / p.P, j = it % p.P;
@@ -358,7 +402,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fused_step_kernel(const __gr
         }
         count_done(C.spec_done + u);
       }
-    } else if ((it -= n_spec) < n_rep) {  // repair
+    } else if (kind_tail == 3) {  // repair (it: unit * R + r)
       kind = 3;
       if (tid == 0) next_ticket = atomicAdd(C.words + kCtlWork, 1u);
       const int u = it / R;
@@ -389,9 +433,8 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fused_step_kernel(const __gr
         }
         count_done(C.rep_done + u);
       }
-    } else {  // LSE merge of (unit, head)
+    } else {  // LSE merge of (unit, head) (it: unit * G + h)
       kind = 5;
-      it -= n_rep;
       const int u = it / p.G, h = it % p.G;
       unsigned flag = 0u;
       if (wait_geq(C.sel_done + u, 1u, C, p.status, sh, &flag)) {
@@ -452,6 +495,8 @@ static cudaError_t launch_fused_t(Params p, const CUtensorMap& kmap, const CUten
   long long grid = static_cast<long long>(per_sm) * sms;
   if (grid > items) grid = items;
   if (grid_out) *grid_out = static_cast<int>(grid);
+  // dependent tickets about two rounds of the grid after their unit's SPEC tickets
+  p.dep_lag = p.P > 0 ? static_cast<int>((2 * grid + p.P - 1) / p.P) : p.units;
   return launch_kernel(fused_step_kernel<D, BS>, dim3(static_cast<unsigned>(grid)), dim3(kFusedThreads), smem, s,
                        priority, kmap, vmap, p);
 }

@@ -69,6 +69,7 @@ struct Params {
   int fchunk_blocks; // blocks per SEL item (multiple of 32, at most 128)
   int fregion;       // bytes of the per-CTA shared-memory union of the fused step
   int rep_items;     // REPAIR items per unit of the fused step: item r repairs missed slots r, r + rep_items, ...
+  int dep_lag;       // units between a unit's SPEC tickets and its REPAIR / COMBINE tickets
   // caller buffers (any may be null when the kernel does not use it)
   const uint16_t* q;        // [B][Hq][d] bf16
   const uint16_t* k_new;    // [B][Hkv][d] bf16 token appended by the fused step (append_kv)

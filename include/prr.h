@@ -147,11 +147,13 @@ typedef struct {
   /* Optional (NULL: off).  prr_decode_step_fused records, for every work item its CTAs
    * run, trace[4i..4i+3] = {start ns, end ns, (SM id << 32) | CTA, kind} (%globaltimer;
    * kind 1 selection chunk, 6 top-K finisher, 4 predictor update, 2 speculative block,
-   * 3 repair item, 5 merge).  Records follow the items' ticket order: units*ceil(maxnb/C)
+   * 3 repair item, 5 merge), i = the item's ticket.  Items: units*ceil(maxnb/C)
    * selection chunks (C blocks each: units*maxnb/512 rounded up to a multiple of 32,
-   * clamped to [32, 128]), units finishers, units predictor updates, units*P speculative
-   * slots, units*R repair items (R = min(K, max(4, ceil(1024/units)))), units*G merges.
-   * Items that did not run stay zero.  Size: 4 * (that many records) words. */
+   * clamped to [32, 128]), units finishers, units predictor updates, units*P
+   * speculative slots, units*R repair items (R = min(K, max(4, ceil(1024/units)))) and
+   * units*G merges; the tickets of a unit's repair items and merges follow its
+   * speculative slots a few units later.  Items that did not run stay zero.  Size:
+   * 4 * (the number of items) words. */
   unsigned long long* trace;
   /* Optional (NULL: off).  Eight counters the step adds to (atomically; the caller
    * zeroes them):  [0] units whose top-K came straight from the 32-block group tie
