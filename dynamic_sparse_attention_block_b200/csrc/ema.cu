@@ -9,6 +9,8 @@ __global__ void __launch_bounds__(256) ema_predict_kernel(const __grid_constant_
   ema_unit(p, blockIdx.x, smem, [] { return true; }, cta_grp());
 }
 
+size_t ema_smem_bytes(int maxnb) { return ema_scratch_bytes(maxnb); }
+
 cudaError_t launch_ema(const Params& p, cudaStream_t s, int priority) {
   const size_t smem = ema_scratch_bytes(p.maxnb);
   cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(ema_predict_kernel));

@@ -17,6 +17,16 @@ using namespace prr;
 
 namespace {
 
+// Shared-memory ceilings of the kernels that keep a unit's per-block state on chip: the
+// selection finisher (keys and bitmaps) and the predictor (the fp64 EMA state).
+constexpr size_t kMaxSmemPerCta = 227 * 1024;
+
+int maxnb_of(const prr_dims* d) { return static_cast<int>((d->cap_tokens + d->bs - 1) / d->bs); }
+
+bool select_fits(const prr_dims* d) { return prr::select_smem_bytes(d->d, maxnb_of(d)) <= kMaxSmemPerCta; }
+
+bool ema_fits(const prr_dims* d) { return prr::ema_smem_bytes(maxnb_of(d)) <= kMaxSmemPerCta; }
+
 constexpr int kVersion = 100;  // 0.1.0
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -301,7 +311,7 @@ prr_status prr_select_topk(const prr_dims* dims, const uint16_t* q, const uint16
                            const int32_t* seq_lens, const int32_t* pred, int32_t* sel,
                            int32_t* missed, int32_t* n_missed, uint8_t* keep, void* ws,
                            cudaStream_t stream) {
-  if (!dims_ok(dims)) return PRR_ERR_SHAPE;
+  if (!dims_ok(dims) || !select_fits(dims)) return PRR_ERR_SHAPE;
   if (!q || !summ || !seq_lens || !sel || !missed || !n_missed || !ws) return PRR_ERR_INVALID_ARG;
   if (dims->P > 0 && (!pred || !keep)) return PRR_ERR_INVALID_ARG;
   if (!aligned16(summ)) return PRR_ERR_INVALID_ARG;
@@ -320,7 +330,7 @@ prr_status prr_select_topk(const prr_dims* dims, const uint16_t* q, const uint16
 prr_status prr_ema_predict(const prr_dims* dims, double* ema, const int32_t* sel,
                            const int32_t* seq_lens, int32_t* pred_next, void* ws,
                            cudaStream_t stream) {
-  if (!dims_ok(dims)) return PRR_ERR_SHAPE;
+  if (!dims_ok(dims) || !ema_fits(dims)) return PRR_ERR_SHAPE;
   if (!ema || !seq_lens || !ws || (dims->P > 0 && !pred_next)) return PRR_ERR_INVALID_ARG;
   Params p = base_params(dims, ws);
   p.ema = ema;
@@ -446,6 +456,7 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* b, void
   Params p;
   const prr_status st = step_params(dims, b, ws, ws_bytes, &p);
   if (st != PRR_OK) return st;
+  if (!select_fits(dims) || !ema_fits(dims)) return PRR_ERR_SHAPE;
   CUtensorMap km, vm;
   if (!make_kv_map(&km, b->k_cache, dims) || !make_kv_map(&vm, b->v_cache, dims)) return PRR_ERR_CUDA;
   const DeviceInfo di = device_info();

@@ -21,9 +21,8 @@
 // tokens, so each warp finishes whole output columns and the tiles are free before the
 // partial is written out.
 //
-// The copies and the arithmetic are separate steps (attn_issue, attn_compute): the
-// standalone kernels run both in one CTA; the fused step's producer warp issues the
-// copies into its ring while a consumer group computes an earlier block.
+// The copies and the arithmetic are separate steps (attn_issue, attn_compute): one
+// thread issues the copies, then the whole CTA computes (block_partial runs both).
 #pragma once
 
 #include "prr_kernels.cuh"

@@ -32,11 +32,10 @@ __device__ __forceinline__ void report(int* status, int code) {
 
 // ------------------------------------------------------------------ thread groups
 //
-// The building blocks below run on a GROUP of threads: a whole CTA (the standalone
-// kernels) or one warp-aligned group of a warp-specialised CTA (the fused step, whose
-// consumer groups of 4 warps synchronise on their own named barrier while the producer
-// warp keeps issuing copies).  tid is the thread's index inside the group, nt the
-// group's size (a multiple of 32), bar the named barrier (0 = the CTA's __syncthreads).
+// The building blocks below run on a GROUP of threads: a whole CTA (every kernel of
+// this library), or a warp-aligned part of one that synchronises on its own named
+// barrier.  tid is the thread's index inside the group, nt the group's size (a
+// multiple of 32), bar the named barrier (0 = the CTA's __syncthreads).
 struct Grp {
   int tid;
   int nt;

@@ -11,10 +11,8 @@
 namespace prr {
 
 #ifdef PRR_PHASE_DEBUG
-// Debug builds only: per-unit phase timestamps of the finisher / predictor, and per
-// fused item {copies issued, K landed, V landed, slot handed back}.
+// Debug builds only: per-unit phase timestamps of the finisher / predictor.
 __device__ unsigned long long g_phase[2][4096][8];
-__device__ unsigned long long g_item[1 << 16][4];
 #define PRR_PHASE(kind, u, k) \
   do {                        \
     if ((threadIdx.x & 127) == 0 && (u) < 4096) g_phase[kind][u][k] = global_ns(); \

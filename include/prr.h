@@ -35,6 +35,12 @@
  *    part_l = sum_i 2^(logit_i - part_m), part_O = sum_i 2^(logit_i - part_m) v_i.
  *  - Supported shapes: d in {64, 128}; bs in {64, 128}; 1 <= G <= 8; 1 <= K <= 128;
  *    0 <= P <= 128; cap_tokens >= 1.  Others return PRR_ERR_SHAPE.
+ *  - Shared-memory ceilings on maxnb = ceil(cap_tokens/bs), checked before anything is
+ *    enqueued (PRR_ERR_SHAPE beyond them): the selection finisher keeps a unit's keys
+ *    and bitmaps on chip, so prr_select_topk, prr_select_topk_static and
+ *    prr_decode_step take maxnb up to 19,715 blocks at d = 128 (34,800 at d = 64); the
+ *    predictor keeps a unit's fp64 EMA state on chip, so prr_ema_predict and both decode
+ *    steps take maxnb up to 26,756 blocks.
  *  - Errors: argument and shape checks happen on the host before anything is
  *    enqueued and return a prr_status.  A failed launch returns PRR_ERR_CUDA.
  *    Problems that only the device can see (a seq_len out of range, a malformed
@@ -290,20 +296,20 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* buf, vo
                            size_t ws_bytes, cudaStream_t select_stream, cudaStream_t spec_stream,
                            const prr_step_events* events);
 
-/* The same decode step (a1-a7) in ONE persistent launch on `stream`: one CTA per SM, a
- * producer warp that keeps the K/V and summary copies of the next items in flight and
- * two consumer groups that compute.  Selection chunks are handed out first, then
- * speculation; the consumer that scores a unit's last chunk runs its top-K at once
- * and queues the unit's repairs and predictor update, and the unit's last partial
- * queues its merges, so no work item waits for another.  A speculative block that
- * selection has already dropped is skipped.  step_parity (0 or 1) must alternate
- * between consecutive calls that share `ws`: each launch uses one copy of the
+/* The same decode step (a1-a7) in ONE persistent launch on `stream`: resident CTAs of
+ * 128 threads (three per SM at the usual shapes) take work items from one counter --
+ * every unit's selection chunks first, then its top-K finishers, predictor updates,
+ * speculative blocks, repairs and merges.  A dependent item waits, bounded, in the CTA
+ * that took it for the items it reads, which always hold lower tickets; a speculative
+ * block that selection has already dropped is skipped.  step_parity (0 or 1) must
+ * alternate between consecutive calls that share `ws`: each launch uses one copy of the
  * workspace control words and clears the other for the next launch.  Same buffers,
  * results and error behaviour as prr_decode_step; capturable in a CUDA graph (one
- * graph per parity).  Size limit: each shared-memory slot must hold the finisher's
- * and the predictor's per-unit scratch, about 12*maxnb bytes, next to two K/V tiles;
- * dims whose slots no longer fit twice in 227 KB (maxnb beyond roughly 12,000 blocks)
- * return PRR_ERR_SHAPE -- prr_decode_step has no such limit below 50,000 blocks.
+ * graph per parity).  Size limit: a CTA's shared memory must hold the predictor's
+ * per-unit scratch (about 7.2 KB + 8.4*maxnb bytes) next to two K/V tiles, within
+ * 227 KB, so maxnb = ceil(cap_tokens/bs) up to 26,756 blocks; beyond that the call
+ * returns PRR_ERR_SHAPE.  Above about 8,000 blocks fewer CTAs fit per SM and the step
+ * slows down.
  * PRR abstract / method summary: speculation overlaps selection and stays off the
  * critical path; repair merges the missed blocks without recomputation. */
 prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* buf, void* ws,

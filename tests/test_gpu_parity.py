@@ -584,3 +584,28 @@ def test_bad_pred_sets_status_without_fault():
     dec.step(to_dev_bits(W.queries(w, 1)[0]))
     torch.cuda.synchronize()
     assert dec.device_status() == 2
+
+
+def test_shape_ceilings_are_refused_before_launch():
+    """Dims beyond a kernel's shared-memory ceiling (include/prr.h: the selection
+    finisher up to 19,715 blocks at d = 128, the predictor and the fused step up to
+    26,756) are refused with PRR_ERR_SHAPE before anything is enqueued; below them both
+    paths run."""
+    from dynamic_sparse_attention_block_b200._abi import PrrError
+    bs = 64
+    # maxnb: (two-stream runs, fused runs)
+    for maxnb, streams_ok, fused_ok in ((19000, True, True), (24000, False, True), (28000, False, False)):
+        dims = prr.Dims(B=1, Hq=4, Hkv=1, d=128, bs=bs, cap_tokens=maxnb * bs, K=8, P=8)
+        dec = prr.PRRDecoder(dims)
+        dec.seq_lens.fill_(4096)
+        q = torch.zeros((1, 4, 128), dtype=torch.bfloat16, device="cuda")
+        for run, ok in ((lambda: dec.step(q), streams_ok), (lambda: dec.step_fused(q), fused_ok)):
+            if ok:
+                run()
+                torch.cuda.synchronize()
+                assert dec.device_status() == 0
+            else:
+                with pytest.raises(PrrError) as err:
+                    run()
+                assert err.value.status == 2, maxnb  # PRR_ERR_SHAPE
+        del dec
