@@ -25,11 +25,11 @@ class PrrDims(ctypes.Structure):
     _fields_ = [("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("d", _i32), ("bs", _i32),
                 ("cap_tokens", _i32), ("K", _i32), ("P", _i32), ("alpha", ctypes.c_double),
                 ("scale", ctypes.c_float), ("selector", _i32), ("n_sink", _i32), ("n_local", _i32),
-                ("pages", _i32), ("block_table", _c_void_p)]
+                ("pages", _i32), ("block_table", _c_void_p), ("n_rep", _i32), ("rep_offsets", _c_void_p)]
 
 
 # block selectors (PRR_SELECT_* in include/prr.h)
-SELECTORS = {"group_sum": 0, "group_max": 1, "per_head": 2}
+SELECTORS = {"group_sum": 0, "group_max": 1, "per_head": 2, "representative": 3}
 
 
 class PrrStepBuffers(ctypes.Structure):
@@ -134,11 +134,13 @@ class Dims:
     P: int
     alpha: float = 0.9
     scale: Optional[float] = None
-    selector: str = "group_sum"   # "group_sum", "group_max" or "per_head"
+    selector: str = "group_sum"   # "group_sum", "group_max", "per_head" or "representative"
     n_sink: int = 0               # forced first blocks
     n_local: int = 0              # forced newest blocks
     pages: int = 0                # paged KV pool size (0: contiguous caches)
     block_table: Optional[int] = None  # device address of the int32 [B][maxnb] block table
+    n_rep: int = 0                # representative tokens per block (representative selector)
+    rep_offsets: Optional[int] = None  # device address of the uint8 [B][Hkv][maxnb][n_rep] offsets
 
     @property
     def G(self) -> int:
@@ -166,7 +168,7 @@ class Dims:
         sc = self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
         return PrrDims(self.B, self.Hq, self.Hkv, self.d, self.bs, self.cap_tokens, self.K,
                        self.P, float(self.alpha), float(sc), SELECTORS[self.selector], self.n_sink, self.n_local,
-                       self.pages, self.block_table)
+                       self.pages, self.block_table, self.n_rep, self.rep_offsets)
 
 
 def _dims(d) -> PrrDims:

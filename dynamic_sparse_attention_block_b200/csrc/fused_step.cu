@@ -239,7 +239,7 @@ __device__ void sel_item(const Params& p, const FusedCtl& C, int u, int chunk, u
                        reinterpret_cast<uint32_t*>(summ_unit + static_cast<size_t>(tail) * 2 * D), lane);
     uint32_t key = 0u;
     if (lane < wrows) {
-      key = block_key(p, first + lane, nb, score_row<D>(p, tile + lane * ROWB, coef, lane));
+      key = block_key(p, first + lane, nb, score_block<D>(p, tile + lane * ROWB, coef, lane, kvu, first + lane, n));
       p.keys[static_cast<size_t>(u) * p.maxnb + first + lane] = key;
     }
     write_group_summary(p, u, first / 32, key, lane < wrows);

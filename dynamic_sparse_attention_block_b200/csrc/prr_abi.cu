@@ -41,7 +41,8 @@ bool dims_ok(const prr_dims* d) {
   if (d->cap_tokens < 1 || d->K < 1 || d->K > 128 || d->P < 0 || d->P > 128) return false;
   if (!(d->alpha >= 0.0 && d->alpha <= 1.0)) return false;
   if (!std::isfinite(d->scale)) return false;
-  if (d->selector < PRR_SELECT_GROUP_SUM || d->selector > PRR_SELECT_PER_HEAD) return false;
+  if (d->selector < PRR_SELECT_GROUP_SUM || d->selector > PRR_SELECT_REPRESENTATIVE) return false;
+  if (d->selector == PRR_SELECT_REPRESENTATIVE && (d->n_rep < 1 || d->n_rep > 16 || !d->rep_offsets)) return false;
   if (d->n_sink < 0 || d->n_sink > (1 << 22) || d->n_local < 0 || d->n_local > (1 << 22)) return false;
   if (d->pages < 0 || (d->pages > 0) != (d->block_table != nullptr)) return false;
   if (static_cast<long long>(d->pages) * d->Hkv >= (1LL << 31)) return false;
@@ -144,6 +145,10 @@ Params base_params(const prr_dims* d, void* ws, bool kv_units = false) {
   p.n_local = d->n_local;
   p.pages = d->pages;
   p.table = d->block_table;
+  if (d->selector == PRR_SELECT_REPRESENTATIVE) {
+    p.rep = d->rep_offsets;
+    p.n_rep = d->n_rep;
+  }
   p.d = d->d;
   p.bs = d->bs;
   p.cap = d->cap_tokens;
@@ -312,6 +317,7 @@ prr_status prr_select_topk(const prr_dims* dims, const uint16_t* q, const uint16
                            int32_t* missed, int32_t* n_missed, uint8_t* keep, void* ws,
                            cudaStream_t stream) {
   if (!dims_ok(dims) || !select_fits(dims)) return PRR_ERR_SHAPE;
+  if (dims->selector == PRR_SELECT_REPRESENTATIVE) return PRR_ERR_SHAPE;  // needs the key cache: the step calls
   if (!q || !summ || !seq_lens || !sel || !missed || !n_missed || !ws) return PRR_ERR_INVALID_ARG;
   if (dims->P > 0 && (!pred || !keep)) return PRR_ERR_INVALID_ARG;
   if (!aligned16(summ)) return PRR_ERR_INVALID_ARG;

@@ -55,6 +55,9 @@ struct Params {
   // paged KV: pools [pages][Hkv][bs][d], table [B][maxnb] block -> page (null: contiguous)
   int pages;
   const int* table;
+  // representative-key selector (null: summary bounds): offsets [units][maxnb][n_rep]
+  const uint8_t* rep;
+  int n_rep;
   float scale_log2;  // softmax scale * log2(e): logits are handled in base 2
   double alpha;      // EMA decay
   int append_summary;  // selection also folds token n-1 into its block summary

@@ -169,10 +169,56 @@ __device__ __forceinline__ float score_summary_row_max(const unsigned char* row,
 // Bytes of the scoring coefficients: one set for the group sum, G sets for the max.
 __host__ __device__ constexpr size_t coef_bytes(int D, int sets) { return static_cast<size_t>(sets) * 2 * (4 * D / 16) * 16; }
 
-// Both variants: coefficients for unit u's query rows qg (group-synchronise before use).
+// Selector variant (representative keys, InfLLM-style): block b is represented by
+// n_rep of its own tokens, offsets rep[(kvu*maxnb + b)*n_rep + j] inside the block (an
+// offset at or past the valid tokens of a ragged tail stands for the last valid one),
+// and scores sum_h sum_j q_h . k_rep_j = sum_j qsum . k_rep_j, qsum = sum_h q_h.  The
+// coefficient area then holds qsum (D floats).  On the dyadic grid every product is a
+// multiple of 1/64 and every partial sum stays below 2^24 units, so the fp32 score is
+// exact in any order.  The key rows are read through L2: the step may have written the
+// appended row in this launch.
+template <int D>
+__device__ __forceinline__ void load_qsum(const Params& p, const uint16_t* qg, float* qs, const Grp& g) {
+  for (int c = g.tid; c < D; c += g.nt) {
+    float acc = 0.f;
+    for (int h = 0; h < p.G; ++h) acc += __uint_as_float(static_cast<uint32_t>(qg[h * D + c]) << 16);
+    qs[c] = acc;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ float score_rep_block(const Params& p, int kvu, int b, int n, const float* qs) {
+  const int valid = min(p.bs, n - b * p.bs);
+  const uint8_t* offs = p.rep + (static_cast<size_t>(kvu) * p.maxnb + b) * p.n_rep;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  for (int j = 0; j < p.n_rep; ++j) {
+    const int off = min(static_cast<int>(offs[j]), valid - 1);
+    const long long row = kv_row(p, kvu, b * p.bs + off);
+    if (row < 0) continue;  // a bad block-table entry (reported by kv_row)
+    const uint4* kr = reinterpret_cast<const uint4*>(p.kc + static_cast<size_t>(row) * D);
+#pragma unroll 4
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+      const uint4 w = __ldcg(kr + c8);
+      const float* q8 = qs + 8 * c8;
+      a0 = fmaf(q8[0], bf16_lo(w.x), a0);
+      a1 = fmaf(q8[2], bf16_lo(w.y), a1);
+      a2 = fmaf(q8[4], bf16_lo(w.z), a2);
+      a3 = fmaf(q8[6], bf16_lo(w.w), a3);
+      a0 = fmaf(q8[1], bf16_hi(w.x), a0);
+      a1 = fmaf(q8[3], bf16_hi(w.y), a1);
+      a2 = fmaf(q8[5], bf16_hi(w.z), a2);
+      a3 = fmaf(q8[7], bf16_hi(w.w), a3);
+    }
+  }
+  return (a0 + a1) + (a2 + a3);
+}
+
+// Every variant: coefficients for unit u's query rows qg (group-synchronise before use).
 template <int D>
 __device__ __forceinline__ void load_coef(const Params& p, const uint16_t* qg, float4* coef, const Grp& g) {
-  if (p.sel_max) {
+  if (p.rep) {
+    load_qsum<D>(p, qg, reinterpret_cast<float*>(coef), g);
+  } else if (p.sel_max) {
     load_head_coef<D>(p, qg, coef, g);
   } else {
     load_group_coef<D>(p, qg, coef, coef + (4 * D / 16), g);
@@ -183,6 +229,15 @@ template <int D>
 __device__ __forceinline__ float score_row(const Params& p, const unsigned char* row, const float4* coef, int lane) {
   if (p.sel_max) return score_summary_row_max<D>(row, coef, p.G, lane);
   return score_summary_row<D>(row, coef, coef + (4 * D / 16), lane);
+}
+
+// The score of block b of KV slice kvu (n tokens): its summary row, or its
+// representative keys under the representative-key selector.
+template <int D>
+__device__ __forceinline__ float score_block(const Params& p, const unsigned char* row, const float4* coef, int lane,
+                                             int kvu, int b, int n) {
+  if (p.rep) return score_rep_block<D>(p, kvu, b, n, reinterpret_cast<const float*>(coef));
+  return score_row<D>(p, row, coef, lane);
 }
 
 // Ranking key of block b (of nb) with score s: forced sink blocks rank above

@@ -99,6 +99,7 @@ extern "C" prr_status prr_select_topk_static(const prr_dims* dims, const uint16_
                                              int32_t* missed, int32_t* n_missed, uint8_t* keep,
                                              int32_t* status, cudaStream_t stream) {
   if (prr_workspace_bytes(dims) == 0) return PRR_ERR_SHAPE;  // same shape rules as the other calls
+  if (dims->selector == PRR_SELECT_REPRESENTATIVE) return PRR_ERR_SHAPE;  // summary selectors only
   if (prr::select_smem_bytes(dims->d, static_cast<int>((dims->cap_tokens + dims->bs - 1) / dims->bs)) >
       227 * 1024)
     return PRR_ERR_SHAPE;  // the finisher's on-chip scratch, as prr_select_topk

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(256, 1) select_topk_kernel(const __grid_consta
                          reinterpret_cast<uint32_t*>(summ_unit + static_cast<size_t>(tail) * 2 * D), lane);
       uint32_t key = 0u;
       if (lane < rows) {
-        key = block_key(p, first + lane, nb, score_row<D>(p, tile + lane * ROWB, coef, lane));
+        key = block_key(p, first + lane, nb, score_block<D>(p, tile + lane * ROWB, coef, lane, kvu, first + lane, n));
         keys_out[first + lane] = key;
       }
       write_group_summary(p, u, first / 32, key, lane < rows);

@@ -27,10 +27,12 @@ class PRRDecoder:
     """
 
     def __init__(self, dims: Dims, device: Optional[torch.device] = None,
-                 block_table: Optional[torch.Tensor] = None):
+                 block_table: Optional[torch.Tensor] = None, rep_offsets: Optional[torch.Tensor] = None):
         """dims.pages > 0 makes the KV cache a paged pool [pages][Hkv][bs][d];
         `block_table` (int32 [B][maxnb], page of block j of sequence b) then defaults to
-        block j of sequence b in page b*maxnb + j."""
+        block j of sequence b in page b*maxnb + j.  The representative-key selector
+        takes `rep_offsets` (uint8 [B][Hkv][maxnb][n_rep], offsets of each block's
+        representative tokens inside the block)."""
         if not torch.cuda.is_available():
             raise RuntimeError("PRRDecoder needs a CUDA device")
         _abi.load()
@@ -49,6 +51,12 @@ class PRRDecoder:
             self.k_cache = torch.zeros((dims.pages, Hkv, dims.bs, d), dtype=torch.bfloat16, device=dev)
         else:
             self.k_cache = torch.zeros((B, Hkv, cap, d), dtype=torch.bfloat16, device=dev)
+        self.rep_offsets = None
+        if dims.selector == "representative":
+            if rep_offsets is None or tuple(rep_offsets.shape) != (B, Hkv, maxnb, dims.n_rep):
+                raise ValueError("the representative selector needs rep_offsets [B][Hkv][maxnb][n_rep]")
+            self.rep_offsets = rep_offsets.to(device=dev, dtype=torch.uint8).contiguous()
+            dims = dataclasses.replace(dims, rep_offsets=self.rep_offsets.data_ptr())
         self.dims = dims
         self.v_cache = torch.zeros_like(self.k_cache)
         self.seq_lens = torch.zeros((B,), dtype=torch.int32, device=dev)

@@ -100,7 +100,14 @@ typedef struct {
    *   PRR_SELECT_PER_HEAD   every query head selects its own top-K with its own bound;
    *                         then a "unit" is a (sequence, query head) pair, and the
    *                         per-unit arrays below are [B][Hq][...] instead of
-   *                         [B][Hkv][...] (summaries and KV stay per KV head). */
+   *                         [B][Hkv][...] (summaries and KV stay per KV head).
+   *   PRR_SELECT_REPRESENTATIVE  one selection per KV head; each block is represented by
+   *                         n_rep of its own tokens (rep_offsets, below; InfLLM-style,
+   *                         the InfLLM title is in PRR's reference list) and scores
+   *                         sum_h sum_j q_h . k_rep_j over the group's query heads.
+   *                         It reads the key cache, so only the decode steps take it;
+   *                         prr_select_topk and prr_select_topk_static return
+   *                         PRR_ERR_SHAPE for it. */
   int32_t selector;
   int32_t n_sink;     /* the first n_sink blocks are always selected (attention sinks), 0..2^22 */
   int32_t n_local;    /* the newest n_local blocks are always selected (local window), 0..2^22;
@@ -117,11 +124,18 @@ typedef struct {
    * that block is not read. */
   int32_t pages;
   const int32_t* block_table;
+  /* PRR_SELECT_REPRESENTATIVE only (otherwise 0 and NULL): n_rep (1..16) representative
+   * tokens per block, and rep_offsets (device uint8 [B][Hkv][maxnb][n_rep]) their
+   * offsets inside the block, chosen when the block was built.  An offset at or past a
+   * ragged tail's valid tokens stands for the block's last valid token. */
+  int32_t n_rep;
+  const uint8_t* rep_offsets;
 } prr_dims;
 
 #define PRR_SELECT_GROUP_SUM 0
 #define PRR_SELECT_GROUP_MAX 1
 #define PRR_SELECT_PER_HEAD 2
+#define PRR_SELECT_REPRESENTATIVE 3
 
 /* Buffers of one decode step (see the shapes above). */
 typedef struct {

@@ -31,12 +31,16 @@ def shuffled_block_table(w: W.Workload, maxnb: int, spare: int, seed: int = 5):
 def make_decoder(w: W.Workload, steps: int, cap_extra: int = 0, paged: bool = False) -> Tuple[PRRDecoder, Dims]:
     cap = w.N0 + steps + cap_extra
     dims = Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, bs=w.bs, cap_tokens=cap, K=w.K, P=w.P,
-                alpha=w.alpha, selector=w.selector, n_sink=w.n_sink, n_local=w.n_local)
+                alpha=w.alpha, selector=w.selector, n_sink=w.n_sink, n_local=w.n_local, n_rep=w.n_rep)
     table = None
     if paged:
         table, pages = shuffled_block_table(w, dims.maxnb, spare=7)
         dims = dataclasses.replace(dims, pages=pages)
-    dec = PRRDecoder(dims, block_table=table)
+    reps = None
+    if w.selector == "representative":
+        reps = torch.from_numpy(np.stack([np.stack([W.rep_offsets(w, b, h, dims.maxnb) for h in range(w.Hkv)])
+                                          for b in range(w.B)]))
+    dec = PRRDecoder(dims, block_table=table, rep_offsets=reps)
     for b in range(w.B):
         for h in range(w.Hkv):
             k0, v0 = W.kv_prefix(w, b, h, w.n0(b))

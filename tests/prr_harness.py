@@ -51,6 +51,7 @@ class UnitOracle:
     ema: np.ndarray
     pred: np.ndarray   # Pred_t (ascending)
     o: OR.Oracle
+    rep: Optional[np.ndarray] = None  # [maxnb][n_rep] representative offsets (representative selector)
 
     @property
     def kv_head(self) -> int:
@@ -77,7 +78,8 @@ class UnitOracle:
         smin[:lo.shape[0]], smax[:lo.shape[0]] = lo, hi
         ema = np.zeros(maxnb)
         pred = o.top_ranked(np.zeros(w.nb(n0)), w.P) if w.P > 0 else np.zeros(0, np.int32)
-        return cls(w, b, kvh, k, v, smin, smax, ema, pred, o)
+        rep = W.rep_offsets(w, b, kv, maxnb) if w.selector == "representative" else None
+        return cls(w, b, kvh, k, v, smin, smax, ema, pred, o, rep)
 
     def select(self, t: int, q_bits: np.ndarray):
         """Summary update for token N0+t, scores, true top-K (all from the oracle)."""
@@ -90,6 +92,8 @@ class UnitOracle:
         qg = f64(q_bits[self.b, self.qrows])
         if w.selector == "group_max":
             s = o.block_scores_max(qg, self.smin[:nb], self.smax[:nb])
+        elif w.selector == "representative":
+            s = o.block_scores_rep(qg, self.k, n, w.bs, self.rep[:nb].astype(np.int32))
         else:  # group sum, or one head's own bound under per-head selection
             s = o.block_scores(qg, self.smin[:nb], self.smax[:nb])
         if w.n_sink or w.n_local:

@@ -364,14 +364,45 @@ def test_decode_full_size_append_in_step():
 @pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("selector,n_sink,n_local", [
     ("group_max", 0, 0), ("per_head", 0, 0), ("group_sum", 2, 3), ("group_max", 1, 4), ("per_head", 1, 2),
+    ("representative", 0, 0), ("representative", 1, 2),
 ])
 def test_decode_selector_variants(mode, selector, n_sink, n_local):
     """The selector variants of the representative DSA methods (group max of the
-    per-head bounds, per-query-head selection, forced sink and local blocks) through
-    both step implementations, every unit, against the oracle's variants."""
+    per-head bounds, per-query-head selection, InfLLM-style representative keys, forced
+    sink and local blocks) through both step implementations, every unit, against the
+    oracle's variants."""
     w = W.workload("tiny").with_(name="variant", B=2, Hq=8, Hkv=2, d=128, N0=3000, bs=64, K=12, P=12, steps=6,
-                                 walk_p=0.8, selector=selector, n_sink=n_sink, n_local=n_local)
+                                 walk_p=0.8, selector=selector, n_sink=n_sink, n_local=n_local,
+                                 n_rep=3 if selector == "representative" else 0)
     _assert_ok(run_parity(w, steps=6, mode=mode))
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_decode_representative_keys_in_step(paged):
+    """The representative-key selector with 128-token blocks, 4 representatives, the
+    token appended inside the fused launch (a representative of the tail block may be
+    the new token) and, paged, its keys read through the block table."""
+    w = W.workload("tiny").with_(name="rep", B=2, Hq=8, Hkv=2, d=128, N0=5000, bs=128, K=8, P=8, steps=5,
+                                 walk_p=0.8, selector="representative", n_rep=4)
+    _assert_ok(run_parity(w, steps=5, append="step", paged=paged))
+
+
+def test_select_topk_refuses_representative_keys():
+    """prr_select_topk takes no key cache, so the representative-key selector is refused
+    there (PRR_ERR_SHAPE) before anything is enqueued."""
+    from dynamic_sparse_attention_block_b200._abi import PrrError
+    reps = torch.zeros((1, 1, 4, 2), dtype=torch.uint8, device="cuda")
+    dims = prr.Dims(B=1, Hq=4, Hkv=1, d=128, bs=64, cap_tokens=256, K=2, P=2, selector="representative", n_rep=2,
+                    rep_offsets=reps.data_ptr())
+    ws = torch.zeros(prr.prr_workspace_bytes(dims), dtype=torch.uint8, device="cuda")
+    t = torch.zeros((1, 1, 2), dtype=torch.int32, device="cuda")
+    with pytest.raises(PrrError) as err:
+        prr.prr_select_topk(dims, torch.zeros((1, 4, 128), dtype=torch.bfloat16, device="cuda"),
+                            torch.zeros((1, 1, 4, 2, 128), dtype=torch.bfloat16, device="cuda"),
+                            torch.full((1,), 200, dtype=torch.int32, device="cuda"), t, t.clone(), t.clone(),
+                            torch.zeros((1, 1), dtype=torch.int32, device="cuda"),
+                            torch.zeros((1, 1, 2), dtype=torch.uint8, device="cuda"), ws)
+    assert err.value.status == 2
 
 
 @pytest.mark.parametrize("selector", ["group_max", "per_head"])

@@ -34,11 +34,11 @@ import numpy as np
 
 __all__ = [
     "Workload", "WORKLOADS", "workload", "f32_to_bf16_bits", "bf16_bits_to_f32",
-    "kv_prefix", "kv_appended", "queries", "forced_prediction", "forced_kept_count",
+    "kv_prefix", "kv_appended", "queries", "forced_prediction", "forced_kept_count", "rep_offsets",
 ]
 
 # stream tags (plain integers so SeedSequence accepts them)
-_TAG_K0, _TAG_V0, _TAG_KNEW, _TAG_VNEW, _TAG_Q, _TAG_FORCED = 11, 12, 13, 14, 15, 16
+_TAG_K0, _TAG_V0, _TAG_KNEW, _TAG_VNEW, _TAG_Q, _TAG_FORCED, _TAG_REP = 11, 12, 13, 14, 15, 16, 17
 
 
 @dataclasses.dataclass(frozen=True)
@@ -63,6 +63,7 @@ class Workload:
     n_sink: int = 0              # forced first blocks
     n_local: int = 0             # forced newest blocks
     n0_seq: Optional[Sequence[int]] = None  # ragged batch: context of each sequence (each <= N0)
+    n_rep: int = 0               # representative tokens per block (selector "representative")
 
     @property
     def G(self) -> int:
@@ -190,6 +191,16 @@ def queries(w: Workload, steps: Optional[int] = None) -> np.ndarray:
                 cur = np.where(keep, cur, fresh)
             out[t, b] = cur
     return out
+
+
+# ----------------------------------------------------------------------------- representatives
+
+def rep_offsets(w: Workload, b: int, kvh: int, maxnb: int) -> np.ndarray:
+    """Offsets [maxnb][n_rep] (uint8, uniform in [0, bs)) of each block's representative
+    tokens for the representative-key selector: an input chosen when a block is built
+    (here seeded per (sequence, KV head)), not part of the method's arithmetic."""
+    rng = _rng(w, b, _TAG_REP, kvh)
+    return rng.integers(0, w.bs, size=(maxnb, w.n_rep), dtype=np.uint8)
 
 
 # ----------------------------------------------------------------------------- forced prediction
