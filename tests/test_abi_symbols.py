@@ -80,3 +80,32 @@ def test_header_compiles_standalone(tmp_path, lang, std):
     r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-Werror", f"-std={std}", "-I", os.path.join(ROOT, "include"),
                         "-I", cuda_inc, str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+@pytest.mark.parametrize("struct,cls", [("prr_dims", "PrrDims"), ("prr_step_buffers", "PrrStepBuffers"),
+                                        ("prr_step_events", "PrrStepEvents")])
+def test_binding_structs_match_the_header_layout(tmp_path, struct, cls):
+    """The ctypes mirrors of the header's structs have the C compiler's layout: every
+    field at the same offset, and the same size."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no host compiler")
+    mirror = getattr(_abi, cls)
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "prr.h"', 'int main(void) {',
+             f'  printf("size %zu\\n", sizeof({struct}));']
+    for name, _ in mirror._fields_:
+        lines.append(f'  printf("{name} %zu\\n", offsetof({struct}, {name}));')
+    lines += ['  return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    r = subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = dict(ln.split() for ln in subprocess.run([str(exe)], capture_output=True, text=True).stdout.splitlines())
+    assert int(out["size"]) == ctypes.sizeof(mirror)
+    for name, _ in mirror._fields_:
+        assert int(out[name]) == getattr(mirror, name).offset, name

@@ -85,3 +85,14 @@ def test_trace_summary_on_a_synthetic_timeline():
     assert s["spec"]["n"] == 1 and s["spec"]["start_min_us"] == 2.0
     assert s["ema"]["n"] == 0 and s["end_us"] == 10.0
     assert s["finish"]["n"] == 1 and s["finisher"] == {"n": 1, "dur_p50_us": 3.0, "dur_max_us": 3.0}
+
+
+def test_rep_offsets_are_seeded_and_in_range():
+    """Representative offsets (an input of the representative-key selector) depend only
+    on the workload's seed, the sequence and the KV head, and lie inside a block."""
+    w = W.workload("tiny").with_(selector="representative", n_rep=4, B=2, Hkv=2, Hq=8)
+    a = W.rep_offsets(w, 1, 1, 70)
+    assert a.shape == (70, 4) and a.dtype == np.uint8
+    assert a.min() >= 0 and a.max() < w.bs
+    assert np.array_equal(a, W.rep_offsets(w, 1, 1, 70))
+    assert not np.array_equal(a, W.rep_offsets(w, 1, 0, 70))
