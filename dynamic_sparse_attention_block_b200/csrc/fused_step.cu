@@ -25,7 +25,8 @@
 // last speculative block.
 //
 // Waits only ever target items with a smaller index, which were taken by CTAs that are
-// already running, so every wait ends without any co-residency assumption.  Each wait
+// already running, so every wait ends without any co-residency assumption.  The counts
+// and the ticket order are defined in prr_schedule.h, which a host test enumerates.  Each wait
 // is bounded (kWaitLimitNs); a timeout records PRR_DEV_WAIT_TIMEOUT and raises an abort
 // flag that makes every later wait give up at once.
 //
@@ -42,26 +43,11 @@
 
 #include "prr_attn.cuh"
 #include "prr_parts.cuh"
+#include "prr_schedule.h"
 
 namespace prr {
 
 constexpr int kFusedThreads = 128;
-constexpr int kFusedChunk = 128;  // most blocks per SEL item (4 warps x 32 rows)
-
-// Blocks per SEL item: a multiple of 32 in [32, 128], about units*maxnb/512, so that a
-// short context still spreads its scan over many CTAs and a long one moves 64 KB per item.
-__host__ __device__ inline int fused_chunk_blocks(int units, int maxnb) {
-  long long c = (static_cast<long long>(units) * maxnb + 511) / 512;
-  c = ((c + 31) / 32) * 32;
-  return static_cast<int>(c < 32 ? 32 : (c > kFusedChunk ? kFusedChunk : c));
-}
-
-// REPAIR items per unit: enough that a unit with many misses spreads them over CTAs,
-// few enough that most items have work.
-inline int fused_rep_items(int units, int K) {
-  const int r = (1024 + units - 1) / units;
-  return std::min(K, std::max(4, r));
-}
 
 // Control words of one copy (word offsets).
 enum : int {
@@ -261,46 +247,6 @@ static __device__ void fin_item(const Params& p, const FusedCtl& C, int u, unsig
   }
 }
 
-// Tickets after the predictor updates (t counts from the first of them), with
-// Lc = min(dep_lag, units) and M = R + G dependent items per unit: first the SPEC
-// tickets of units 0..Lc-1 (P each); then, for k = 0..units-Lc-1, the SPEC tickets of
-// unit Lc+k followed by unit k's R REPAIR and G COMBINE tickets; last the dependent
-// tickets of units units-Lc..units-1.  Every dependent ticket comes after all of its
-// unit's SPEC tickets.  Returns false for a SPEC ticket (*idx = unit * P + slot), true
-// for a dependent one (*kind 3 with *idx = unit * R + r, or 5 with *idx = unit * G + h).
-__device__ __forceinline__ bool decode_tail(const Params& p, int t, int U, int R, int* idx, int* kind) {
-  const int P = p.P, M = R + p.G;
-  const int Lc = min(p.dep_lag, U);
-  int v, r;  // unit and index of a dependent ticket
-  if (t < Lc * P) {
-    *idx = t;
-    return false;
-  }
-  t -= Lc * P;
-  const int mid = (U - Lc) * (P + M);
-  if (t < mid) {
-    const int k = t / (P + M), q = t % (P + M);
-    if (q < P) {
-      *idx = (Lc + k) * P + q;
-      return false;
-    }
-    v = k;
-    r = q - P;
-  } else {
-    t -= mid;
-    v = U - Lc + t / M;
-    r = t % M;
-  }
-  if (r < R) {
-    *kind = 3;
-    *idx = v * R + r;
-  } else {
-    *kind = 5;
-    *idx = v * p.G + (r - R);
-  }
-  return true;
-}
-
 // ---------------------------------------------------------------- the kernel
 template <int D, int BS>
 __global__ void __launch_bounds__(kFusedThreads, 3) fused_step_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -371,7 +317,7 @@ __global__ void __launch_bounds__(kFusedThreads, 3) fused_step_kernel(const __gr
       kind = 4;
       ema_unit(p, it, smem, [&] { return wait_geq(C.sel_done + it, 1u, C, p.status, sh); }, cta_grp());
       count_tail(p, C);
-    } else if (!decode_tail(p, it - n_ema, U, R, &it, &kind_tail)) {  // speculation
+    } else if (!decode_tail(p.P, p.G, p.dep_lag, it - n_ema, U, R, &it, &kind_tail)) {  // speculation
       kind = 2;
       if (tid == 0) next_ticket = atomicAdd(C.words + kCtlWork, 1u);
       const int u = it / p.P, j = it % p.P;
@@ -491,12 +437,12 @@ static cudaError_t launch_fused_t(Params p, const CUtensorMap& kmap, const CUten
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_step_kernel<D, BS>, kFusedThreads, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  const long long items = static_cast<long long>(p.units) * (p.fchunks + 1 + 1 + p.P + p.rep_items + p.G);
+  const long long items = fused_total_items(p.units, p.fchunks, p.P, p.rep_items, p.G);
   long long grid = static_cast<long long>(per_sm) * sms;
   if (grid > items) grid = items;
   if (grid_out) *grid_out = static_cast<int>(grid);
   // dependent tickets about two rounds of the grid after their unit's SPEC tickets
-  p.dep_lag = p.P > 0 ? static_cast<int>((2 * grid + p.P - 1) / p.P) : p.units;
+  p.dep_lag = fused_dep_lag(grid, p.P, p.units);
   return launch_kernel(fused_step_kernel<D, BS>, dim3(static_cast<unsigned>(grid)), dim3(kFusedThreads), smem, s,
                        priority, kmap, vmap, p);
 }
