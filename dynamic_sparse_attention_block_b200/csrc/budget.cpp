@@ -2,8 +2,8 @@
 //
 // PRR sizes its speculation from profiling (PRR abstract: a profiling-guided
 // speculation budget keeps speculative work off the critical path).  Its
-// limitations list says the overheads between profiled grid points come from
-// polynomial regressions in the context length.  So a budget model here is:
+// limitations list says the overheads at context lengths off the profiled grid
+// (between or beyond its points) come from polynomial regressions in the context length.  So a budget model here is:
 //   select_us(x) and, for every profiled budget p_j, spec_us_j(x),
 // each a least-squares polynomial in x = context_tokens / 65536 (a scale that keeps
 // the normal equations well conditioned at 4K-1M tokens).  The budget for a context

@@ -331,7 +331,8 @@ prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* b
 
 /* Profiling-guided speculation budget (PRR abstract: the speculation budget comes from
  * profiling and keeps speculative work off the critical path; limitations: overheads
- * at context lengths between the profiled points come from polynomial regressions).
+ * at context lengths off the profiled grid, between or beyond its points, come from
+ * polynomial regressions).
  * Host functions: they touch no device memory and need no GPU.
  *
  * prr_budget_fit: least-squares polynomial of degree `degree` (0..3) through the n

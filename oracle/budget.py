@@ -2,8 +2,8 @@
 
 TEST INFRASTRUCTURE ONLY, like the rest of this package.  PRR (abstract) sizes its
 speculation from profiling so that speculative work stays off the critical path; its
-limitations list says overheads between profiled context lengths come from polynomial
-regressions.  Reference definitions:
+limitations list says overheads at context lengths off the profiled grid (between or
+beyond its points) come from polynomial regressions.  Reference definitions:
   fit:    least-squares polynomial of the measured times in x = context / 65536
           (numpy's lstsq on the Vandermonde matrix), coefficients lowest order first;
   choose: the largest profiled budget whose predicted speculation time is at most the

@@ -109,3 +109,28 @@ def test_binding_structs_match_the_header_layout(tmp_path, struct, cls):
     assert int(out["size"]) == ctypes.sizeof(mirror)
     for name, _ in mirror._fields_:
         assert int(out[name]) == getattr(mirror, name).offset, name
+
+
+def test_readme_c_example_compiles(tmp_path):
+    """The C example in README.md names only entry points, fields and constants that the
+    header declares, with the right argument counts (it compiles as C99 inside a
+    function that declares the buffers it uses)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no host compiler")
+    text = open(os.path.join(ROOT, "README.md")).read()
+    blocks = re.findall(r"```c\n(.*?)```", text, flags=re.S)
+    assert len(blocks) == 1, "expected one C example"
+    body = [ln for ln in blocks[0].splitlines() if not ln.startswith("#include")]
+    decls = ("  uint16_t *k_cache = 0, *summ = 0; const int32_t *tok_begin = 0, *tok_end = 0;\n"
+             "  int32_t *seq_lens = 0, *pred = 0; int32_t n0 = 0; double *ema = 0; void *ws = 0;\n"
+             "  cudaStream_t stream = 0; int steps = 1; prr_step_buffers buf = {0};\n")
+    src = tmp_path / "example.c"
+    src.write_text('#include "prr.h"\nint example(void) {\n' + decls + "\n".join("  " + ln for ln in body)
+                   + "\n  return 0;\n}\n")
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-Werror", "-Wno-unused-variable", "-std=c99",
+                        "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr + src.read_text()
