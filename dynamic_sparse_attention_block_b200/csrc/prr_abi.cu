@@ -38,7 +38,8 @@ bool dims_ok(const prr_dims* d) {
   if (G > 8) return false;
   if (d->d != 64 && d->d != 128) return false;
   if (d->bs != 64 && d->bs != 128) return false;
-  if (d->cap_tokens < 1 || d->K < 1 || d->K > 128 || d->P < 0 || d->P > 128) return false;
+  if (d->cap_tokens < 1 || d->cap_tokens > (1 << 30)) return false;  // ceil(cap/bs) stays in int
+  if (d->K < 1 || d->K > 128 || d->P < 0 || d->P > 128) return false;
   if (!(d->alpha >= 0.0 && d->alpha <= 1.0)) return false;
   if (!std::isfinite(d->scale)) return false;
   if (d->selector < PRR_SELECT_GROUP_SUM || d->selector > PRR_SELECT_REPRESENTATIVE) return false;

@@ -34,7 +34,9 @@
  *    Partials use base-2 logits: part_m = max_i scale*log2(e)*q.k_i over the block,
  *    part_l = sum_i 2^(logit_i - part_m), part_O = sum_i 2^(logit_i - part_m) v_i.
  *  - Supported shapes: d in {64, 128}; bs in {64, 128}; 1 <= G <= 8; 1 <= K <= 128;
- *    0 <= P <= 128; cap_tokens >= 1.  Others return PRR_ERR_SHAPE.
+ *    0 <= P <= 128; 1 <= cap_tokens <= 2^30; at most 65,535 selection units (B*Hkv, or
+ *    B*Hq under PRR_SELECT_PER_HEAD); pages*Hkv below 2^31.  Others return
+ *    PRR_ERR_SHAPE (prr_workspace_bytes returns 0).
  *  - Shared-memory ceilings on maxnb = ceil(cap_tokens/bs), checked before anything is
  *    enqueued (PRR_ERR_SHAPE beyond them): the selection finisher keeps a unit's keys
  *    and bitmaps on chip, so prr_select_topk, prr_select_topk_static and

@@ -49,6 +49,22 @@ def test_host_side_calls(lib):
     assert _abi.prr_workspace_bytes(bad) == 0  # unsupported head dim
 
 
+@pytest.mark.parametrize("kw,ok", [
+    (dict(cap_tokens=1 << 30), True), (dict(cap_tokens=(1 << 30) + 1), False), (dict(cap_tokens=2**31 - 1), False),
+    (dict(B=8191, Hkv=8, Hq=32), True), (dict(B=8192, Hkv=8, Hq=32), False),  # 65,535 selection units
+    (dict(B=2047, Hkv=8, Hq=32, selector="per_head"), True), (dict(B=2048, Hkv=8, Hq=32, selector="per_head"), False),
+    (dict(K=128, P=128), True), (dict(K=129), False), (dict(P=129), False), (dict(P=-1), False),
+    (dict(Hq=64, Hkv=8), True), (dict(Hq=72, Hkv=8), False), (dict(Hq=12, Hkv=8), False),  # 1 <= G <= 8
+    (dict(bs=32), False), (dict(d=256), False),
+])
+def test_shape_rules(lib, kw, ok):
+    """The documented shape rules, at and just past each bound: a refused shape sizes no
+    workspace (0 bytes)."""
+    base = dict(B=1, Hq=32, Hkv=8, d=128, bs=64, cap_tokens=4096, K=64, P=64)
+    base.update(kw)
+    assert (_abi.prr_workspace_bytes(_abi.Dims(**base)) > 0) == ok, kw
+
+
 def test_argument_checks_return_before_any_launch(lib):
     d = _abi.Dims(B=1, Hq=4, Hkv=1, d=64, bs=64, cap_tokens=4096, K=8, P=8).c()
     null = ctypes.c_void_p(0)
