@@ -298,11 +298,13 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": nsteps, "warmup": args.warmup, "ms_per_step": sps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(workload_config(w, args), l2="not applicable (host CPU)"),
+        "config": workload_config(w, args),  # the GPU arm's config, key for key
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                          "sample": f"{nsteps} full oracle decode steps ({units} (sequence, KV head) "
                                    f"units each) of {w.name}, OpenMP over units",
-                         "cpu_model": cpu_model()},
+                         "cpu_model": cpu_model(),
+                         "caches": "no flush between steps on the host; each step streams the "
+                                   "whole KV cache, which is far larger than the host caches"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     if nsteps < args.steps:

@@ -78,3 +78,23 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
     args = argparse.Namespace(workload="tiny", warmup=3, steps=2, gpus=2, ref_budget_s=1.0)
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_carries_the_gpu_arm_config(monkeypatch, capsys):
+    """The reference arm prints one JSON line with the same metric, unit, direction and
+    config as the GPU arm, so the two lines compare like for like."""
+    import json
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    args = argparse.Namespace(workload="tiny", warmup=3, steps=2, gpus=1, ref_budget_s=5.0, batch=0)
+    assert bench.run_reference(args) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.workload_config(bench.base_workload(args), args)
+    assert (line["metric"], line["unit"], line["higher_is_better"]) == (bench.METRIC, bench.UNIT, True)
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["value"] > 0 and line["steps"] >= 1
