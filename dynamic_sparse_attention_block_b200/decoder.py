@@ -189,15 +189,24 @@ class PRRDecoder:
 
     def prefill(self, k: Optional[torch.Tensor], v: Optional[torch.Tensor], n0) -> None:
         """Start decoding after an initial context: optionally copy it in (k, v
-        [B][Hkv][n0][d] bf16, contiguous caches only; else load_context wrote it), set the
-        sequence lengths (n0: one length, or one per sequence), build all block
-        summaries, reset the EMA and predict from the zero state."""
+        [B][Hkv][n][d] bf16 with n >= every length, contiguous caches only; else
+        load_context wrote it), set the sequence lengths (n0: one length, or one per
+        sequence), build all block summaries, reset the EMA and predict from the zero
+        state."""
         d = self.dims
         lens = [int(n0)] * d.B if isinstance(n0, int) else [int(x) for x in n0]
+        if len(lens) != d.B or min(lens) < 1 or max(lens) > d.cap_tokens:
+            raise ValueError(f"need {d.B} lengths in [1, {d.cap_tokens}], got {lens}")
+        if k is not None:
+            if self.block_table is not None:
+                raise ValueError("prefill copies k/v into a contiguous cache only: fill a paged one with load_context")
+            if v is None or k.shape != v.shape or k.dim() != 4 or k.shape[2] < max(lens):
+                raise ValueError("k and v must both be [B][Hkv][n][d] with n >= every sequence length")
         with torch.cuda.stream(self.select_stream):
             if k is not None:
-                self.k_cache[:, :, :lens[0]].copy_(k)
-                self.v_cache[:, :, :lens[0]].copy_(v)
+                n = k.shape[2]
+                self.k_cache[:, :, :n].copy_(k)
+                self.v_cache[:, :, :n].copy_(v)
             self.seq_lens.copy_(torch.tensor(lens, dtype=torch.int32))
             self.ema.zero_()
             self.pred_buf.fill_(-1)
@@ -245,11 +254,19 @@ class PRRDecoder:
                            self.ws, stream or self.select_stream)
 
     # ------------------------------------------------------------------ the step
+    def _after_caller(self, st) -> None:
+        """Order `st` after the caller's current stream, on which the step's input
+        tensors were produced (a no-op when the caller already runs on `st`)."""
+        cur = torch.cuda.current_stream(self.device)
+        if cur != st:
+            st.wait_stream(cur)
+
     def step(self, q: Optional[torch.Tensor] = None, timing: Optional[dict] = None,
              swap: bool = True, append: bool = False) -> None:
         """One decode step on the state's streams (q [B][Hq][d] bf16 is copied into the
         step's query buffer first when given).  Swaps Pred_t / Pred_{t+1} afterwards."""
         if q is not None:
+            self._after_caller(self.select_stream)
             with torch.cuda.stream(self.select_stream):
                 self.q.copy_(q)
         _abi.prr_decode_step(self.dims, self.buffers(append=append), self.ws, self.select_stream,
@@ -264,6 +281,8 @@ class PRRDecoder:
         With k_new / v_new ([B][Hkv][d] bf16, copied into the decoder's token buffers)
         or `append`, the launch also appends the step's token (no separate append)."""
         st = stream or self.select_stream
+        if q is not None or k_new is not None:
+            self._after_caller(st)
         with torch.cuda.stream(st):
             if q is not None:
                 self.q.copy_(q)
@@ -289,7 +308,7 @@ def summarize_trace(trace) -> dict:
     started and the last ended (microseconds after the earliest start), and the p50 /
     mean / max item duration; "finisher" repeats the count and durations of the top-K
     finisher items.  `trace` is the [records][4] array of prr_step_buffers (start ns,
-    end ns, SM << 32 | group << 16 | CTA, kind)."""
+    end ns, SM << 32 | CTA index, kind)."""
     import numpy as np
     tr = np.asarray(trace, dtype=np.int64)
     ran = tr[:, 0] > 0

@@ -79,13 +79,12 @@ class ShardedDecoder:
 
     def step_fused(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor) -> None:
         """One decode step on every local shard: q [B][Hq][d], k_new / v_new [B][Hkv][d]
-        bf16 (full batch, any device); each shard takes its own sequences' rows and
-        appends its token inside its fused launch."""
+        bf16 (full batch, any device); each shard copies its own sequences' rows on its
+        step stream (after the caller's current stream) and appends its token inside
+        its fused launch."""
         for (b0, b1), dec in self.shards:
-            dev = dec.device
-            with torch.cuda.device(dev):
-                dec.step_fused(q[b0:b1].to(dev, non_blocking=True), k_new=k_new[b0:b1].to(dev, non_blocking=True),
-                               v_new=v_new[b0:b1].to(dev, non_blocking=True))
+            with torch.cuda.device(dec.device):
+                dec.step_fused(q[b0:b1], k_new=k_new[b0:b1], v_new=v_new[b0:b1])
 
     def outputs(self) -> List[Tuple[Tuple[int, int], torch.Tensor, torch.Tensor]]:
         """(sequence range, out, lse) of every local shard, on its own device."""
