@@ -1,8 +1,9 @@
 """Profiling-guided speculation budget.
 
 PRR (abstract) sizes its speculative work from profiling so that it stays off the
-critical path; its limitations list says the overheads at context lengths between the
-profiled ones come from polynomial regressions.  This module:
+critical path; its limitations list says the overheads at context lengths off the
+profiled grid (between or beyond its points) come from polynomial regressions.  This
+module:
 
 - profiles, on the GPU, the selection time and the speculation time over a grid of
   context lengths and speculation budgets: of the two-stream decode step

@@ -249,9 +249,11 @@ class PRRDecoder:
         self.select_stream.synchronize()
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
-        """Write the step's token (k_new/v_new [B][Hkv][d] bf16) and advance seq_lens."""
-        _abi.prr_append_kv(self.dims, k_new, v_new, self.seq_lens, self.k_cache, self.v_cache,
-                           self.ws, stream or self.select_stream)
+        """Write the step's token (k_new/v_new [B][Hkv][d] bf16) and advance seq_lens, on
+        `stream` (default: the step stream, ordered after the caller's current stream)."""
+        st = stream or self.select_stream
+        self._after_caller(st)
+        _abi.prr_append_kv(self.dims, k_new, v_new, self.seq_lens, self.k_cache, self.v_cache, self.ws, st)
 
     # ------------------------------------------------------------------ the step
     def _after_caller(self, st) -> None:
