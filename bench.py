@@ -285,6 +285,22 @@ def oracle_run(w: W.Workload, warmup: int, steps: int, budget_s: float, nthreads
     return tokens / secs, secs / max(len(times), 1), len(times), w.units, used
 
 
+def cpu_baseline(w: W.Workload, args, caches=None) -> dict:
+    """The oracle's step on all host cores (OpenMP over units), timed on a bounded sample
+    of the workload after 2 warm-up steps, and its rate on one thread (one cold step).
+    `caches` needs room for 2 + args.cpu_max_steps tokens after N0."""
+    threads = os.cpu_count() or 1
+    value, sps, nsteps, units, used = oracle_run(w, 2, args.cpu_max_steps, args.cpu_budget_s, threads,
+                                                 caches=caches)
+    v1, sps1, _, _, used1 = oracle_run(w, 0, 1, 0.0, 1, caches=caches)
+    return {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{nsteps} oracle decode steps of {w.name} after 2 warm-up steps "
+                      f"({units} units per step, ~{args.cpu_budget_s:.0f} s budget)",
+            "cpu_model": cpu_model(),
+            "single_thread": {"value": v1, "unit": UNIT, "cores": used1, "ms_per_step": sps1 * 1e3,
+                              "sample": f"1 oracle decode step of {w.name} on one thread"}}
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -644,13 +660,7 @@ def run_gpu(args):
     cpu_steps = 2 + args.cpu_max_steps
     caches = host_cache(w, w.N0 + (cpu_steps if rank == 0 and world == 1 and not args.no_cpu_baseline else 0))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        threads = os.cpu_count() or 1
-        value, sps, nsteps, units, used = oracle_run(w, 2, args.cpu_max_steps, args.cpu_budget_s, threads,
-                                                     caches=caches)
-        cpu = {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
-               "sample": f"{nsteps} oracle decode steps of {w.name} after 2 warm-up steps "
-                         f"({units} units per step, ~{args.cpu_budget_s:.0f} s budget)",
-               "cpu_model": cpu_model()}
+        cpu = cpu_baseline(w, args, caches)
         # the oracle appended its own tokens past N0; the GPU run reads only [0, N0)
 
     head, tokens, secs, step_ms = measure(w, args, hbm_peak, e2e=not args.no_e2e,

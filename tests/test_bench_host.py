@@ -88,3 +88,14 @@ def test_kernel_source_sha_covers_every_kernel_source():
     assert "fused_step.cu" in names and "prr_schedule.h" in names
     sha = bench.kernel_source_sha()
     assert len(sha) == 16 and sha == bench.kernel_source_sha()
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    import argparse
+    w = W.workload("tiny")
+    args = argparse.Namespace(cpu_max_steps=3, cpu_budget_s=5.0)
+    r = bench.cpu_baseline(w, args, caches=bench.host_cache(w, w.N0 + 2 + args.cpu_max_steps))
+    assert r["kind"] == "oracle" and r["unit"] == bench.UNIT and r["value"] > 0
+    assert r["cores"] >= 1 and r["cpu_model"]
+    one = r["single_thread"]
+    assert one["cores"] == 1 and one["value"] > 0 and one["ms_per_step"] > 0
