@@ -202,6 +202,7 @@ class PRRDecoder:
                 raise ValueError("prefill copies k/v into a contiguous cache only: fill a paged one with load_context")
             if v is None or k.shape != v.shape or k.dim() != 4 or k.shape[2] < max(lens):
                 raise ValueError("k and v must both be [B][Hkv][n][d] with n >= every sequence length")
+        self._after_caller(self.select_stream)  # k/v (or load_context's writes) come from the caller's stream
         with torch.cuda.stream(self.select_stream):
             if k is not None:
                 n = k.shape[2]
@@ -237,6 +238,7 @@ class PRRDecoder:
     def restore(self, ck: dict) -> None:
         """Load a checkpoint() into this decoder (same dims): the next step continues
         exactly where the checkpointed decoder stopped."""
+        self._after_caller(self.select_stream)
         with torch.cuda.stream(self.select_stream):
             for name in ("k_cache", "v_cache", "seq_lens", "summ", "ema"):
                 getattr(self, name).copy_(ck[name])
