@@ -3,7 +3,7 @@ and through the fp64 oracle, step by step, and collect a comparison report."""
 from __future__ import annotations
 
 import dataclasses
-from typing import Dict, Iterable, List, Optional, Sequence, Tuple
+from typing import Dict, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
