@@ -69,20 +69,6 @@ __device__ __forceinline__ bool gsync_and(const Grp& g, bool v) {
   return r != 0;
 }
 
-__device__ __forceinline__ bool gsync_or(const Grp& g, bool v) {
-  if (g.bar == 0) return __syncthreads_or(v) != 0;
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "r"(g.bar), "r"(g.nt)
-      : "memory");
-  return r != 0;
-}
-
 // Add to an optional step counter (thread-level; callers pick one thread).
 __device__ __forceinline__ void bump(unsigned long long* stats, int which, unsigned long long v = 1ull) {
   if (stats) atomicAdd(stats + which, v);
@@ -112,13 +98,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
-// Plain arrival (no transaction bytes): completes a phase of a count-1 barrier that
-// carries no copy.  Release semantics: earlier writes of this thread are visible to
-// threads that observe the phase completion.
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   uint32_t ok;
   asm volatile(
@@ -129,22 +108,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
       : "r"(smem_addr(bar)), "r"(phase)
       : "memory");
   return ok != 0;
-}
-
-// The same wait for a thread that has nothing else to do: after the first failed
-// probes it backs off, so that a waiting warp leaves the issue slots to the warps of
-// the SM that compute.
-__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t phase, int* status) {
-  if (mbar_try_wait(bar, phase)) return true;
-  const uint64_t t0 = global_ns();
-  for (int spin = 0; !mbar_try_wait(bar, phase); ++spin) {
-    if (spin > 4) __nanosleep(64);
-    if (global_ns() - t0 > kWaitLimitNs) {
-      report(status, kDevWaitTimeout);
-      return false;
-    }
-  }
-  return true;
 }
 
 // Wait for the barrier's phase to complete, giving up after kWaitLimitNs.  On time-out
@@ -205,23 +168,9 @@ __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void st_release64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_relaxed64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned long long ld_acquire64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 
@@ -232,29 +181,6 @@ __device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
   unsigned old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
-}
-
-// Atomic add at GPU scope with release semantics only (returns the old value): the
-// caller's earlier writes are ordered before it, and later accesses need not wait for
-// it, so its result can be used well after it was issued.
-__device__ __forceinline__ unsigned atom_add_release(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
-__device__ __forceinline__ unsigned long long ld_relaxed64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
 }
 
 // Hint: start bringing `bytes` (multiple of 16, 16-byte aligned) of global memory into L2.
@@ -288,18 +214,6 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// transpose of an 8x8 b16 matrix held one row-pair per thread (fragment layout)
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
