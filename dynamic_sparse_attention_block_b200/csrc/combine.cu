@@ -12,7 +12,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ Pa
 
 cudaError_t launch_combine(const Params& p, cudaStream_t s, int priority) {
   const dim3 grid(p.G, p.units);
-  const size_t smem = combine_scratch_bytes(p.P, p.K, p.d);
+  const size_t smem = combine_scratch_bytes(p.P, p.d);
   if (p.d == 128) return launch_kernel(combine_kernel<128>, grid, dim3(128), smem, s, priority, p);
   return launch_kernel(combine_kernel<64>, grid, dim3(128), smem, s, priority, p);
 }

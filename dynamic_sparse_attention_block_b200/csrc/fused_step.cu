@@ -407,7 +407,7 @@ static size_t fused_region_bytes(const Params& p) {
   size_t r = sel_aux_offset<D>(p) + group_coef_bytes<D>(p) + 2 * D;
   r = std::max(r, AttnTile<D, BS>::bytes);
   r = std::max(r, ema_scratch_bytes(p.maxnb));
-  r = std::max(r, combine_scratch_bytes(p.P, p.K, D));
+  r = std::max(r, combine_scratch_bytes(p.P, D));
   return (r + 15) & ~static_cast<size_t>(15);
 }
 

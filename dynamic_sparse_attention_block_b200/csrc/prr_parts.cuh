@@ -658,7 +658,7 @@ __device__ inline void ema_unit(const Params& p, int u, unsigned char* scratch, 
 // speculative slots are folded first; `wait_repair()` (CTA-uniform) runs between the
 // two phases, so a caller can start on the speculative part before repair is done.
 
-__host__ __device__ constexpr size_t combine_scratch_bytes(int P, int K, int D) {
+__host__ __device__ constexpr size_t combine_scratch_bytes(int P, int D) {
   return static_cast<size_t>(P) * 12 + 16 * 4 + 4 * static_cast<size_t>(D) * 4 + 64;
 }
 
