@@ -103,3 +103,50 @@ def test_two_gloo_shards_gather_the_whole_batch():
     full = _oracle_step(w, 0, w.B, steps=3)
     for r in range(world):  # every rank holds the whole batch, in sequence order
         assert np.array_equal(got[r][0], full["out"]) and np.array_equal(got[r][1], full["lse"])
+
+
+class _FakeShard:
+    """Stands in for PRRDecoder in the host-logic test: records the rows it is given."""
+
+    def __init__(self, dims, dev):
+        self.dims, self.given, self.calls = dims, dev, []
+        self.device = -1  # torch.cuda.device(-1) is a no-op, so no GPU is touched
+        self.out = torch.zeros((dims.B, dims.Hq, dims.d))
+        self.lse = torch.zeros((dims.B, dims.Hq))
+
+    def step_fused(self, q, k_new, v_new):
+        self.calls.append((q.clone(), k_new.clone(), v_new.clone()))
+
+
+def test_sharded_decoder_hands_each_shard_its_own_rows():
+    from dynamic_sparse_attention_block_b200 import Dims
+    from dynamic_sparse_attention_block_b200.sharding import ShardedDecoder
+    dims = Dims(B=5, Hq=4, Hkv=2, d=64, bs=64, cap_tokens=128, K=2, P=2)
+    made = []
+
+    def make(d, dev):
+        made.append(_FakeShard(d, dev))
+        return made[-1]
+
+    sh = ShardedDecoder(dims, devices=["gpu0", "gpu1", "gpu2"], make=make)  # one process, three GPUs
+    assert [(f.dims.B, f.given) for f in made] == [(2, "gpu0"), (2, "gpu1"), (1, "gpu2")]
+    q = torch.arange(5 * 4 * 64, dtype=torch.float32).view(5, 4, 64)
+    kn = torch.arange(5 * 2 * 64, dtype=torch.float32).view(5, 2, 64)
+    vn = -kn
+    sh.step_fused(q, kn, vn)
+    for (b0, b1), f in sh.shards:
+        (gq, gk, gv), = f.calls
+        assert torch.equal(gq, q[b0:b1]) and torch.equal(gk, kn[b0:b1]) and torch.equal(gv, vn[b0:b1])
+    assert [rng for rng, _, _ in sh.outputs()] == [(0, 2), (2, 4), (4, 5)]
+
+    # one process per GPU: rank 1 of 3 builds only its own shard
+    made.clear()
+    one = ShardedDecoder(dims, devices=["mine"], rank=1, world=3, make=make)
+    assert [rng for rng, _ in one.shards] == [(2, 4)] and made[0].given == "mine"
+    # a batch smaller than the world leaves empty shards out
+    made.clear()
+    small = ShardedDecoder(Dims(B=1, Hq=4, Hkv=2, d=64, bs=64, cap_tokens=128, K=2, P=2),
+                           devices=["a", "b"], make=make)
+    assert len(small.shards) == 1 and len(made) == 1
+    with pytest.raises(ValueError):
+        ShardedDecoder(dims, devices=["a", "b"], world=3, make=make)
