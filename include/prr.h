@@ -206,7 +206,8 @@ typedef struct {
   cudaEvent_t t_ema_end;     /* spec_stream: after the predictor */
 } prr_step_events;
 
-/* Library version (major*10000 + minor*100 + patch). */
+/* Library version (major*10000 + minor*100 + patch).  Library plumbing, like the
+ * status, workspace and append calls below: no passage of the pages defines them. */
 int prr_version(void);
 
 /* Human-readable name of a status. */
@@ -236,7 +237,8 @@ prr_status prr_get_device_status(const void* ws, int32_t* code);
 
 /* Write one new token per (sequence, KV head): k_new/v_new [B][Hkv][d] go to position
  * seq_lens[b] of the caches, then seq_lens[b] is incremented (a full cache leaves
- * seq_lens unchanged and sets PRR_DEV_BAD_SEQ_LEN). */
+ * seq_lens unchanged and sets PRR_DEV_BAD_SEQ_LEN).  The pages take the decode loop's
+ * one-token-per-step cache growth as given; this is that step, not part of PRR. */
 prr_status prr_append_kv(const prr_dims* dims, const uint16_t* k_new, const uint16_t* v_new,
                          int32_t* seq_lens, uint16_t* k_cache, uint16_t* v_cache, void* ws,
                          cudaStream_t stream);
@@ -345,10 +347,11 @@ prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* b
 prr_status prr_budget_fit(const double* context_tokens, const double* us, int32_t n, int32_t degree,
                           double* coef);
 
-/* prr_budget_choose: the speculation budget for a context of context_tokens: the largest
- * p_grid[j] whose predicted speculation time (polynomial spec_coef[j], [np][degree+1])
- * does not exceed the predicted selection time (polynomial sel_coef, [degree+1]), or 0
- * if none does.  p_grid must be strictly ascending.  *p_out receives the budget. */
+/* prr_budget_choose (same passages as prr_budget_fit): the speculation budget for a
+ * context of context_tokens: the largest p_grid[j] whose predicted speculation time
+ * (polynomial spec_coef[j], [np][degree+1]) does not exceed the predicted selection
+ * time (polynomial sel_coef, [degree+1]), or 0 if none does.  p_grid must be strictly
+ * ascending.  *p_out receives the budget. */
 prr_status prr_budget_choose(const double* sel_coef, const double* spec_coef, const int32_t* p_grid,
                              int32_t np, int32_t degree, int32_t context_tokens, int32_t* p_out);
 
