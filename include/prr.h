@@ -38,11 +38,15 @@
  *    B*Hq under PRR_SELECT_PER_HEAD); pages*Hkv below 2^31.  Others return
  *    PRR_ERR_SHAPE (prr_workspace_bytes returns 0).
  *  - Shared-memory ceilings on maxnb = ceil(cap_tokens/bs), checked before anything is
- *    enqueued (PRR_ERR_SHAPE beyond them): the selection finisher keeps a unit's keys
- *    and bitmaps on chip, so prr_select_topk, prr_select_topk_static and
- *    prr_decode_step take maxnb up to 19,715 blocks at d = 128 (34,800 at d = 64); the
- *    predictor keeps a unit's fp64 EMA state on chip, so prr_ema_predict and both decode
- *    steps take maxnb up to 26,756 blocks.
+ *    enqueued (PRR_ERR_SHAPE beyond them), all within 227 KB per CTA:
+ *    - the selection finisher keeps a unit's keys and bitmaps on chip, so
+ *      prr_select_topk, prr_select_topk_static and prr_decode_step take maxnb up to
+ *      19,715 blocks at d = 128 (34,800 at d = 64);
+ *    - the predictor keeps a unit's fp64 EMA state on chip (7,232 bytes plus 8 per
+ *      block plus 12 per 32 blocks), so prr_ema_predict and prr_decode_step take maxnb
+ *      up to 26,890 blocks;
+ *    - prr_decode_step_fused holds the same predictor state plus 1,080 bytes of its
+ *      own (alignment slack and barriers), so it takes maxnb up to 26,760 blocks.
  *  - Errors: argument and shape checks happen on the host before anything is
  *    enqueued and return a prr_status.  A failed launch returns PRR_ERR_CUDA.
  *    Problems that only the device can see (a seq_len out of range, a malformed
@@ -323,11 +327,11 @@ prr_status prr_decode_step(const prr_dims* dims, const prr_step_buffers* buf, vo
  * alternate between consecutive calls that share `ws`: each launch uses one copy of the
  * workspace control words and clears the other for the next launch.  Same buffers,
  * results and error behaviour as prr_decode_step; capturable in a CUDA graph (one
- * graph per parity).  Size limit: a CTA's shared memory must hold the predictor's
- * per-unit scratch (about 7.2 KB + 8.4*maxnb bytes) next to two K/V tiles, within
- * 227 KB, so maxnb = ceil(cap_tokens/bs) up to 26,756 blocks; beyond that the call
- * returns PRR_ERR_SHAPE.  Above about 8,000 blocks fewer CTAs fit per SM and the step
- * slows down.
+ * graph per parity).  Size limit: a CTA's shared memory holds one item's scratch at a
+ * time, at long contexts the predictor's per-unit state (about 7.1 KB + 8.4 bytes per
+ * block), within 227 KB, so maxnb = ceil(cap_tokens/bs) up to 26,760 blocks;
+ * beyond that the call returns PRR_ERR_SHAPE.  Above about 8,000 blocks fewer CTAs fit
+ * per SM and the step slows down.
  * PRR abstract / method summary: speculation overlaps selection and stays off the
  * critical path; repair merges the missed blocks without recomputation. */
 prr_status prr_decode_step_fused(const prr_dims* dims, const prr_step_buffers* buf, void* ws,

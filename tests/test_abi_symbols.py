@@ -150,3 +150,43 @@ def test_readme_c_example_compiles(tmp_path):
     r = subprocess.run([cc, "-fsyntax-only", "-Wall", "-Werror", "-Wno-unused-variable", "-std=c99",
                         "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr + src.read_text()
+
+
+def _ceiling_call(lib, call, d, maxnb):
+    """Status of `call` with maxnb blocks and never-dereferenced buffer addresses."""
+    dims = _abi.Dims(B=1, Hq=4, Hkv=1, d=d, bs=64, cap_tokens=maxnb * 64, K=8, P=8).c()
+    fake, null = ctypes.c_void_p(1 << 20), ctypes.c_void_p(0)
+    if call == "select":
+        return lib.prr_select_topk(ctypes.byref(dims), fake, fake, fake, fake, fake, fake, fake, fake, fake, null)
+    if call == "static":
+        return lib.prr_select_topk_static(ctypes.byref(dims), fake, fake, fake, fake, fake, fake, fake, fake,
+                                          null, null)
+    if call == "ema":
+        return lib.prr_ema_predict(ctypes.byref(dims), fake, fake, fake, fake, fake, null)
+    buf = _abi.PrrStepBuffers()
+    for i, (name, _) in enumerate(buf._fields_):  # distinct 16-byte-aligned addresses
+        if name not in ("k_new", "v_new", "trace", "stats"):
+            setattr(buf, name, (1 << 20) * (i + 1))
+    big = ctypes.c_size_t(1 << 60)  # workspace size: never the limiting check here
+    if call == "fused":
+        return lib.prr_decode_step_fused(ctypes.byref(dims), ctypes.byref(buf), fake, big, 0, null)
+    ev = _abi.PrrStepEvents()
+    for i, name in enumerate(_abi.STEP_EVENTS):
+        setattr(ev, name, (1 << 20) * (i + 1))
+    return lib.prr_decode_step(ctypes.byref(dims), ctypes.byref(buf), fake, big, null, null, ctypes.byref(ev))
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="at a ceiling the call goes on to launch, which needs real buffers")
+@pytest.mark.parametrize("call,d,limit", [
+    ("select", 128, 19715), ("select", 64, 34800), ("static", 128, 19715), ("static", 64, 34800),
+    ("ema", 128, 26890), ("ema", 64, 26890), ("streams", 128, 19715), ("streams", 64, 26890),
+    ("fused", 128, 26760), ("fused", 64, 26760),
+])
+def test_shared_memory_ceilings_are_the_documented_ones(lib, call, d, limit):
+    """The ceilings include/prr.h states, to the block: one block more is refused with
+    PRR_ERR_SHAPE before anything is enqueued; at the ceiling the call passes every
+    check and only fails on reaching the CUDA runtime (PRR_ERR_CUDA: no GPU here)."""
+    assert f"{limit:,}" in open(HEADER).read()
+    assert _ceiling_call(lib, call, d, limit + 1) == 2
+    assert _ceiling_call(lib, call, d, limit) == 4

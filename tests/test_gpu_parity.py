@@ -619,9 +619,9 @@ def test_bad_pred_sets_status_without_fault():
 
 def test_shape_ceilings_are_refused_before_launch():
     """Dims beyond a kernel's shared-memory ceiling (include/prr.h: the selection
-    finisher up to 19,715 blocks at d = 128, the predictor and the fused step up to
-    26,756) are refused with PRR_ERR_SHAPE before anything is enqueued; below them both
-    paths run."""
+    finisher up to 19,715 blocks at d = 128, the predictor up to 26,890, the fused step
+    up to 26,760) are refused with PRR_ERR_SHAPE before anything is enqueued; below them
+    both paths run."""
     from dynamic_sparse_attention_block_b200._abi import PrrError
     bs = 64
     # maxnb: (two-stream runs, fused runs)
