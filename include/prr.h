@@ -43,8 +43,9 @@
  *      prr_select_topk, prr_select_topk_static and prr_decode_step take maxnb up to
  *      19,715 blocks at d = 128 (34,800 at d = 64);
  *    - the predictor keeps a unit's fp64 EMA state on chip (7,232 bytes plus 8 per
- *      block plus 12 per 32 blocks), so prr_ema_predict and prr_decode_step take maxnb
- *      up to 26,890 blocks;
+ *      block plus 12 per 32 blocks), so prr_ema_predict takes maxnb up to 26,890
+ *      blocks, and prr_decode_step the smaller of its two limits (19,715 at d = 128,
+ *      26,890 at d = 64);
  *    - prr_decode_step_fused holds the same predictor state plus 1,080 bytes of its
  *      own (alignment slack and barriers), so it takes maxnb up to 26,760 blocks.
  *  - Errors: argument and shape checks happen on the host before anything is
