@@ -355,7 +355,7 @@ prr_status prr_speculate(const prr_dims* dims, const uint16_t* q, const uint16_t
   if (dims->P == 0) return PRR_OK;
   if (!q || !k_cache || !v_cache || !seq_lens || !pred || !part_m || !part_l || !part_O || !ws)
     return PRR_ERR_INVALID_ARG;
-  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(part_O)) return PRR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(part_O)) return PRR_ERR_INVALID_ARG;
   Params p = base_params(dims, ws);
   p.q = q;
   p.kc = k_cache;
@@ -380,7 +380,7 @@ prr_status prr_repair_merge(const prr_dims* dims, const uint16_t* q, const uint1
   if (!q || !k_cache || !v_cache || !seq_lens || !missed || !n_missed || !out || !lse || !ws)
     return PRR_ERR_INVALID_ARG;
   if (dims->P > 0 && (!keep || !pred || !part_m || !part_l || !part_O)) return PRR_ERR_INVALID_ARG;
-  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PRR_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PRR_ERR_INVALID_ARG;
   if (part_O && !aligned16(part_O)) return PRR_ERR_INVALID_ARG;
   Params p = base_params(dims, ws);
   p.q = q;

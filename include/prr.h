@@ -15,6 +15,10 @@
  *    allocates, frees or synchronises device memory; only prr_get_device_status
  *    synchronises (to read the status word back).
  *  - bf16 arrays are passed as uint16_t bit patterns.
+ *  - Alignment: q where a call attends with it (prr_speculate, prr_repair_merge and
+ *    both decode steps), and k_cache, v_cache, summ, part_O, out, k_new and v_new
+ *    wherever a call takes them, start on a 16-byte boundary; otherwise the call
+ *    returns PRR_ERR_INVALID_ARG before enqueuing anything.
  *  - Shapes (row-major, innermost last), with units = B*Hkv (B*Hq under
  *    PRR_SELECT_PER_HEAD), G = Hq/Hkv, maxnb = ceil(cap_tokens/bs):
  *      q            [B][Hq][d]               bf16   query of the step

@@ -190,3 +190,50 @@ def test_shared_memory_ceilings_are_the_documented_ones(lib, call, d, limit):
     assert f"{limit:,}" in open(HEADER).read()
     assert _ceiling_call(lib, call, d, limit + 1) == 2
     assert _ceiling_call(lib, call, d, limit) == 4
+
+
+# (entry point, argument position, name) of every buffer a call needs 16-byte aligned.
+_ALIGNED = {
+    "prr_append_kv": (8, [(1, "k_new"), (2, "v_new"), (4, "k_cache"), (5, "v_cache")]),
+    "prr_update_summaries": (9, [(1, "k_cache"), (6, "summ")]),
+    "prr_select_topk": (11, [(2, "summ")]),
+    "prr_select_topk_static": (11, [(2, "summ")]),
+    "prr_speculate": (11, [(1, "q"), (2, "k_cache"), (3, "v_cache"), (8, "part_O")]),
+    "prr_repair_merge": (16, [(1, "q"), (2, "k_cache"), (3, "v_cache"), (11, "part_O"), (12, "out")]),
+}
+
+
+@pytest.mark.parametrize("fn", sorted(_ALIGNED))
+def test_misaligned_buffers_are_refused_before_anything_is_enqueued(lib, fn):
+    """Every buffer that include/prr.h requires on a 16-byte boundary, moved 2 bytes off
+    it, makes the call return PRR_ERR_INVALID_ARG (never-dereferenced addresses; the
+    refusal comes before any CUDA call, so this runs with or without a GPU)."""
+    nargs, aligned = _ALIGNED[fn]
+    dims = _abi.Dims(B=1, Hq=4, Hkv=1, d=64, bs=64, cap_tokens=4096, K=8, P=8).c()
+    for pos, name in aligned:
+        args = [ctypes.byref(dims)] + [ctypes.c_void_p((1 << 20) * (i + 1)) for i in range(1, nargs - 1)]
+        args.append(ctypes.c_void_p(0))  # stream
+        if fn == "prr_update_summaries":
+            args[5] = ctypes.c_int32(1)  # max_range_tokens
+        if fn == "prr_select_topk_static":
+            args[9] = ctypes.c_void_p(0)  # optional status
+        args[pos] = ctypes.c_void_p(args[pos].value + 2)
+        assert getattr(lib, fn)(*args) == 1, (fn, name)
+
+
+def test_misaligned_step_buffers_are_refused(lib):
+    dims = _abi.Dims(B=1, Hq=4, Hkv=1, d=64, bs=64, cap_tokens=4096, K=8, P=8).c()
+    fake = ctypes.c_void_p(1 << 20)
+    big = ctypes.c_size_t(1 << 60)
+    ev = _abi.PrrStepEvents()
+    for i, name in enumerate(_abi.STEP_EVENTS):
+        setattr(ev, name, (1 << 20) * (i + 1))
+    for name in ("q", "k_cache", "v_cache", "summ", "part_O", "out", "k_new", "v_new"):
+        buf = _abi.PrrStepBuffers()
+        for i, (field, _) in enumerate(buf._fields_):
+            if field not in ("trace", "stats"):
+                setattr(buf, field, (1 << 20) * (i + 1))
+        setattr(buf, name, getattr(buf, name) + 2)
+        assert lib.prr_decode_step_fused(ctypes.byref(dims), ctypes.byref(buf), fake, big, 0, None) == 1, name
+        assert lib.prr_decode_step(ctypes.byref(dims), ctypes.byref(buf), fake, big, None, None,
+                                   ctypes.byref(ev)) == 1, name
