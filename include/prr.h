@@ -15,6 +15,10 @@
  *    allocates, frees or synchronises device memory; only prr_get_device_status
  *    synchronises (to read the status word back).
  *  - bf16 arrays are passed as uint16_t bit patterns.
+ *  - NULL: every buffer a call takes is required (PRR_ERR_INVALID_ARG if NULL) except
+ *    where its description says otherwise; with P = 0 (no speculation budget) the
+ *    predicted-slot buffers (pred, pred_next, keep, part_m, part_l, part_O) may be
+ *    NULL, and prr_speculate returns PRR_OK without doing anything.
  *  - Alignment: q where a call attends with it (prr_speculate, prr_repair_merge and
  *    both decode steps), and k_cache, v_cache, summ, part_O, out, k_new and v_new
  *    wherever a call takes them, start on a 16-byte boundary; otherwise the call

@@ -237,3 +237,108 @@ def test_misaligned_step_buffers_are_refused(lib):
         assert lib.prr_decode_step_fused(ctypes.byref(dims), ctypes.byref(buf), fake, big, 0, None) == 1, name
         assert lib.prr_decode_step(ctypes.byref(dims), ctypes.byref(buf), fake, big, None, None,
                                    ctypes.byref(ev)) == 1, name
+
+
+# (entry point, argument count, positions that must not be NULL, positions needed only
+# when P > 0).  Positions count from 0 = dims; the last argument is the stream.
+_REQUIRED = {
+    "prr_append_kv": (8, [1, 2, 3, 4, 5, 6], []),
+    "prr_update_summaries": (9, [1, 6, 7], []),
+    "prr_select_topk": (11, [1, 2, 3, 5, 6, 7, 9], [4, 8]),
+    "prr_select_topk_static": (11, [1, 2, 3, 5, 6, 7], [4, 8]),
+    "prr_ema_predict": (7, [1, 3, 5], [4]),
+    "prr_speculate": (11, [1, 2, 3, 4, 5, 6, 7, 8, 9], []),
+    "prr_repair_merge": (16, [1, 2, 3, 4, 5, 6, 12, 13, 14], [7, 8, 9, 10, 11]),
+}
+
+
+def _args(fn, nargs, dims):
+    args = [ctypes.byref(dims)] + [ctypes.c_void_p((1 << 20) * (i + 1)) for i in range(1, nargs - 1)]
+    args.append(ctypes.c_void_p(0))
+    if fn == "prr_update_summaries":
+        args[5] = ctypes.c_int32(1)
+    if fn == "prr_select_topk_static":
+        args[9] = ctypes.c_void_p(0)
+    return args
+
+
+@pytest.mark.parametrize("fn", sorted(_REQUIRED))
+def test_null_required_buffers_are_refused(lib, fn):
+    """A NULL where include/prr.h needs a buffer returns PRR_ERR_INVALID_ARG before
+    anything is enqueued; buffers of the speculative slots are needed only when P > 0."""
+    nargs, always, with_p = _REQUIRED[fn]
+    for P in (8, 0):
+        dims = _abi.Dims(B=1, Hq=4, Hkv=1, d=64, bs=64, cap_tokens=4096, K=8, P=P).c()
+        needed = always + (with_p if P > 0 else [])
+        if fn == "prr_speculate" and P == 0:
+            needed = []  # nothing to speculate: the call returns PRR_OK at once
+            args = [ctypes.byref(dims)] + [ctypes.c_void_p(0)] * (nargs - 1)
+            assert getattr(lib, fn)(*args) == 0
+        for pos in needed:
+            args = _args(fn, nargs, dims)
+            args[pos] = ctypes.c_void_p(0)
+            assert getattr(lib, fn)(*args) == 1, (fn, P, pos)
+
+
+def test_summary_range_arguments(lib):
+    """prr_update_summaries: tok_begin and tok_end come together; without them the call
+    covers the token just appended, so it needs seq_lens and max_range_tokens = 1; the
+    range bound lies in [1, cap_tokens]."""
+    dims = _abi.Dims(B=1, Hq=4, Hkv=1, d=64, bs=64, cap_tokens=4096, K=8, P=8).c()
+
+    def call(tb, te, sl, mr):
+        args = _args("prr_update_summaries", 9, dims)
+        args[2], args[3], args[4], args[5] = tb, te, sl, ctypes.c_int32(mr)
+        return lib.prr_update_summaries(*args)
+
+    a, null = ctypes.c_void_p(1 << 24), ctypes.c_void_p(0)
+    assert call(a, null, a, 1) == 1 and call(null, a, a, 1) == 1  # one without the other
+    assert call(null, null, null, 1) == 1                          # appended token needs seq_lens
+    assert call(null, null, a, 2) == 2                             # appended token is one token
+    assert call(a, a, null, 0) == 2 and call(a, a, null, 4097) == 2
+
+
+def test_step_argument_rules(lib):
+    """The decode steps: pred and pred_next must differ, the workspace must be at least
+    prr_workspace_bytes, k_new and v_new come together, step_parity is 0 or 1, and the
+    two-stream step needs its four ordering events."""
+    d = _abi.Dims(B=1, Hq=4, Hkv=1, d=64, bs=64, cap_tokens=4096, K=8, P=8)
+    dims = d.c()
+    need = _abi.prr_workspace_bytes(d)
+    ws = ctypes.c_void_p(1 << 20)
+
+    def buffers(**change):
+        buf = _abi.PrrStepBuffers()
+        for i, (field, _) in enumerate(buf._fields_):
+            if field not in ("k_new", "v_new", "trace", "stats"):
+                setattr(buf, field, (1 << 24) * (i + 1))
+        for k, v in change.items():
+            setattr(buf, k, v)
+        return buf
+
+    def events(drop=None):
+        ev = _abi.PrrStepEvents()
+        for i, name in enumerate(_abi.STEP_EVENTS):
+            setattr(ev, name, None if name == drop else (1 << 20) * (i + 1))
+        return ev
+
+    def fused(buf, nbytes=1 << 60, parity=0):
+        return lib.prr_decode_step_fused(ctypes.byref(dims), ctypes.byref(buf), ws, ctypes.c_size_t(nbytes),
+                                         parity, None)
+
+    def streams(buf, nbytes=1 << 60, ev=None):
+        return lib.prr_decode_step(ctypes.byref(dims), ctypes.byref(buf), ws, ctypes.c_size_t(nbytes), None, None,
+                                   ctypes.byref(ev or events()))
+
+    same = buffers()
+    same.pred_next = same.pred
+    assert fused(same) == 1 and streams(same) == 1
+    assert fused(buffers(), nbytes=need - 1) == 3 and streams(buffers(), nbytes=need - 1) == 3
+    half = buffers(k_new=1 << 30)
+    assert fused(half) == 1 and streams(half) == 1
+    assert fused(buffers(), parity=2) == 1 and fused(buffers(), parity=-1) == 1
+    for name in _abi.STEP_EVENTS:
+        assert streams(buffers(), ev=events(drop=name)) == 1, name
+    for field in ("q", "k_cache", "v_cache", "seq_lens", "summ", "ema", "sel", "missed", "n_missed", "out", "lse",
+                  "pred", "pred_next", "keep", "part_m", "part_l", "part_O"):
+        assert fused(buffers(**{field: None})) == 1, field
