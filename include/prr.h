@@ -139,10 +139,11 @@ typedef struct {
    * that block is not read. */
   int32_t pages;
   const int32_t* block_table;
-  /* PRR_SELECT_REPRESENTATIVE only (otherwise 0 and NULL): n_rep (1..16) representative
-   * tokens per block, and rep_offsets (device uint8 [B][Hkv][maxnb][n_rep]) their
-   * offsets inside the block, chosen when the block was built.  An offset at or past a
-   * ragged tail's valid tokens stands for the block's last valid token. */
+  /* PRR_SELECT_REPRESENTATIVE only (the other selectors ignore them): n_rep (1..16)
+   * representative tokens per block, and rep_offsets (device uint8
+   * [B][Hkv][maxnb][n_rep]) their offsets inside the block, chosen when the block was
+   * built.  An offset at or past a ragged tail's valid tokens stands for the block's
+   * last valid token. */
   int32_t n_rep;
   const uint8_t* rep_offsets;
 } prr_dims;

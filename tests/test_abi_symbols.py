@@ -56,6 +56,16 @@ def test_host_side_calls(lib):
     (dict(K=128, P=128), True), (dict(K=129), False), (dict(P=129), False), (dict(P=-1), False),
     (dict(Hq=64, Hkv=8), True), (dict(Hq=72, Hkv=8), False), (dict(Hq=12, Hkv=8), False),  # 1 <= G <= 8
     (dict(bs=32), False), (dict(d=256), False),
+    (dict(selector="representative", n_rep=1, rep_offsets=1 << 20), True),
+    (dict(selector="representative", n_rep=16, rep_offsets=1 << 20), True),
+    (dict(selector="representative", n_rep=17, rep_offsets=1 << 20), False),
+    (dict(selector="representative", n_rep=0, rep_offsets=1 << 20), False),
+    (dict(selector="representative", n_rep=4), False),  # no offsets
+    (dict(n_sink=1 << 22, n_local=1 << 22), True), (dict(n_sink=(1 << 22) + 1), False),
+    (dict(n_local=-1), False), (dict(alpha=1.0), True), (dict(alpha=1.5), False), (dict(alpha=-0.1), False),
+    (dict(pages=64, block_table=1 << 20), True), (dict(pages=64), False),  # a pool needs its table
+    (dict(block_table=1 << 20), False),                                     # and a table its pool
+    (dict(pages=(1 << 28), Hkv=8, Hq=32, block_table=1 << 20), False),      # pages*Hkv reaches 2^31
 ])
 def test_shape_rules(lib, kw, ok):
     """The documented shape rules, at and just past each bound: a refused shape sizes no
