@@ -42,6 +42,9 @@ MUTANTS = [
     ("paged_wrong_head", "((size_t)table[t / bs] * Hkv + h) * bs", "((size_t)table[t / bs] * Hkv) * bs"),
     ("paged_block_not_mapped", "((size_t)table[t / bs] * Hkv + h) * bs", "((size_t)(t / bs) * Hkv + h) * bs"),
     ("rep_tail_not_clamped", "if (off > valid - 1) off = valid - 1;", "if (off > bs - 1) off = bs - 1;"),
+    ("rep_first_head_only", "total += q[h * d + c] * bf16_val(krow[c]);", "total += q[c] * bf16_val(krow[c]);"),
+    ("rep_last_token_only", "for (int j = 0; j < r; ++j) {\n                int off = rep",
+     "for (int j = r - 1; j < r; ++j) {\n                int off = rep"),
 ]
 
 
