@@ -45,6 +45,15 @@ MUTANTS = [
     ("rep_first_head_only", "total += q[h * d + c] * bf16_val(krow[c]);", "total += q[c] * bf16_val(krow[c]);"),
     ("rep_last_token_only", "for (int j = 0; j < r; ++j) {\n                int off = rep",
      "for (int j = r - 1; j < r; ++j) {\n                int off = rep"),
+    ("step_tail_summary_skipped",
+     "oracle_block_summary(ku, n, d, bs, tail, mn + (size_t)tail * d, mx + (size_t)tail * d);", ";"),
+    ("step_predicts_before_update",
+     "oracle_ema_update(e, nb, su, nsel, D->alpha);\n        for (int j = 0; j < D->P; ++j) pn[j] = -1;\n"
+     "        oracle_top_ranked(e, nb, D->P, pn);",
+     "for (int j = 0; j < D->P; ++j) pn[j] = -1;\n        oracle_top_ranked(e, nb, D->P, pn);\n"
+     "        oracle_ema_update(e, nb, su, nsel, D->alpha);"),
+    ("step_wrong_query_group", "qg[h * d + c] = bf16_val(q[((size_t)b * D->Hq + kvh * G + h) * d + c]);",
+     "qg[h * d + c] = bf16_val(q[((size_t)b * D->Hq + h) * d + c]);"),
 ]
 
 
