@@ -52,6 +52,9 @@ MUTANTS = [
      "        oracle_top_ranked(e, nb, D->P, pn);",
      "for (int j = 0; j < D->P; ++j) pn[j] = -1;\n        oracle_top_ranked(e, nb, D->P, pn);\n"
      "        oracle_ema_update(e, nb, su, nsel, D->alpha);"),
+    ("prr_reuses_dropped_partials", "if (!keep[j]) continue;", "if (0 && !keep[j]) continue;"),
+    ("prr_repair_skipped", "for (int i = 0; i < nm; ++i) {\n        oracle_block_partial",
+     "for (int i = 0; i < 0; ++i) {\n        oracle_block_partial"),
     ("step_wrong_query_group", "qg[h * d + c] = bf16_val(q[((size_t)b * D->Hq + kvh * G + h) * d + c]);",
      "qg[h * d + c] = bf16_val(q[((size_t)b * D->Hq + h) * d + c]);"),
 ]
