@@ -96,3 +96,25 @@ def test_rep_offsets_are_seeded_and_in_range():
     assert a.min() >= 0 and a.max() < w.bs
     assert np.array_equal(a, W.rep_offsets(w, 1, 1, 70))
     assert not np.array_equal(a, W.rep_offsets(w, 1, 0, 70))
+
+
+# The benchmarked configurations: (B, Hq, Hkv, d, N0, bs, K, P, steps, q/k kind, walk p)
+CONFIGS = {
+    "tiny": (1, 4, 1, 64, 4096, 64, 8, 8, 16, "grid", 0.9),
+    "llama8b_32k": (1, 32, 8, 128, 32768, 64, 64, 64, 128, "grid", 0.9),
+    "batched_128k": (16, 32, 8, 128, 131072, 128, 32, 32, 64, "grid", 0.9),
+    "repair_sweep_64k": (8, 32, 8, 128, 65536, 64, 64, 64, 32, "gauss", 0.9),
+    "long_512k": (4, 64, 8, 128, 524288, 128, 64, 64, 32, "grid", 0.8),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_workload_shapes_are_the_benchmarked_configs(name):
+    w = W.workload(name)
+    got = (w.B, w.Hq, w.Hkv, w.d, w.N0, w.bs, w.K, w.P, w.steps, w.qk, w.walk_p)
+    assert got == CONFIGS[name]
+    assert w.nb(w.N0 + 1) == -(-(w.N0 + 1) // w.bs)
+    if name == "repair_sweep_64k":  # six forced predictor-overlap levels
+        assert tuple(w.forced_overlaps) == (1.0, 0.97, 0.9, 0.75, 0.5, 0.0)
+    if name == "batched_128k":
+        assert w.per_seq_seed  # seed = b per sequence
