@@ -35,6 +35,11 @@ __global__ void __launch_bounds__(128) update_summaries_kernel(const __grid_cons
     return;
   }
   if (begin == end) return;
+  // a range longer than the call's max_range_tokens touches more blocks than the grid has
+  if ((end - 1) / p.bs - begin / p.bs >= static_cast<int>(gridDim.x)) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) report(p.status, kDevBadRange);
+    return;
+  }
   const int blk = begin / p.bs + blockIdx.x;
   const int t0 = blk * p.bs;
   const int lo_t = max(begin, t0), hi_t = min(end, t0 + p.bs);

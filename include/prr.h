@@ -93,7 +93,7 @@ typedef enum {
 #define PRR_DEV_BAD_PRED 2     /* predicted list entry out of range or not ascending */
 #define PRR_DEV_BAD_MISSED 3   /* missed list entry out of range */
 #define PRR_DEV_WAIT_TIMEOUT 4 /* a bounded wait for a TMA copy gave up */
-#define PRR_DEV_BAD_RANGE 5    /* summary update range outside [0, cap_tokens], or a block-table entry outside [0, pages) */
+#define PRR_DEV_BAD_RANGE 5    /* summary update range outside [0, cap_tokens] or longer than max_range_tokens, or a block-table entry outside [0, pages) */
 
 typedef struct {
   int32_t B;          /* sequences */
@@ -263,7 +263,8 @@ prr_status prr_append_kv(const prr_dims* dims, const uint16_t* k_new, const uint
  * inside a block is folded into the stored summary of that block's earlier tokens.
  * tok_begin/tok_end are device int32 [B]; both NULL means "the token just appended":
  * [seq_lens[b]-1, seq_lens[b]).  max_range_tokens bounds tok_end-tok_begin over all
- * sequences (it sizes the grid).  Summary per Quest (Query-Aware Sparsity for
+ * sequences (it sizes the grid); a longer range sets PRR_DEV_BAD_RANGE and leaves that
+ * sequence's summaries as they were.  Summary per Quest (Query-Aware Sparsity for
  * Efficient Long-Context LLM Inference, in the PRR reference list). */
 prr_status prr_update_summaries(const prr_dims* dims, const uint16_t* k_cache,
                                 const int32_t* tok_begin, const int32_t* tok_end,
