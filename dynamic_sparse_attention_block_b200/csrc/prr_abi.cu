@@ -277,6 +277,8 @@ prr_status prr_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) {
 prr_status prr_get_device_status(const void* ws, int32_t* code) {
   if (!ws || !code) return PRR_ERR_INVALID_ARG;
   int32_t v = 0;
+  // every call that may still write the word can run on any stream, blocking or not
+  if (cudaDeviceSynchronize() != cudaSuccess) return PRR_ERR_CUDA;
   if (cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return PRR_ERR_CUDA;
   *code = v;
   return v == 0 ? PRR_OK : PRR_ERR_DEVICE_STATUS;

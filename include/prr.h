@@ -245,8 +245,10 @@ size_t prr_workspace_bytes(const prr_dims* dims);
  * The kernels leave their tickets re-armed, so steady-state calls need no reset. */
 prr_status prr_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
 
-/* Synchronously read the workspace status word into *code (0 = no error). Returns
- * PRR_OK if the code is 0, PRR_ERR_DEVICE_STATUS otherwise. */
+/* Wait for all work on the current device (cudaDeviceSynchronize, whatever streams the
+ * calls ran on), then read the workspace status word into *code (0 = no error).
+ * Returns PRR_OK if the code is 0, PRR_ERR_DEVICE_STATUS otherwise, PRR_ERR_CUDA if the
+ * wait or the copy fails.  Not for use while a stream capture is in progress. */
 prr_status prr_get_device_status(const void* ws, int32_t* code);
 
 /* Write one new token per (sequence, KV head): k_new/v_new [B][Hkv][d] go to position
